@@ -1,0 +1,667 @@
+// api.cu -- the extern "C" entry points of minf.h: argument checks, workspace
+// carving, TMA descriptors, and the launch sequence of each operation.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace minf {
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(MINF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ workspace
+constexpr size_t kAlign = 256;
+
+struct Carver {
+    char *base;
+    size_t off;
+    explicit Carver(void *b, size_t start) : base(static_cast<char *>(b)), off(start) {}
+    template <class T>
+    T *take(size_t count) {
+        off = (off + kAlign - 1) & ~(kAlign - 1);
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += count * sizeof(T);
+        return p;
+    }
+};
+
+int qtiles(int n) { return (n + kTileM - 1) / kTileM; }
+
+// Vertical-Slash estimate: key chunking for about two CTAs per SM.
+void vs_est_geometry(int n, int n_pairs, int *n_chunks, int *chunk_tiles, int *n_ktiles) {
+    const int kt = (n + 127) / 128;
+    int want = (296 + n_pairs - 1) / std::max(1, n_pairs);
+    want = std::max(1, std::min(want, kt));
+    const int ct = (kt + want - 1) / want;
+    *n_ktiles = kt;
+    *chunk_tiles = ct;
+    *n_chunks = (kt + ct - 1) / ct;
+}
+
+VsEstBufs carve_vs_est(Carver &c, int n, int n_heads, int n_pairs) {
+    VsEstBufs b{};
+    vs_est_geometry(n, n_pairs, &b.n_chunks, &b.chunk_tiles, &b.n_ktiles);
+    int maxc = 0, ct, kt;
+    vs_est_geometry(n, 1, &maxc, &ct, &kt);  // upper bound of n_chunks over pairings
+    b.part = c.take<float2>((size_t)n_heads * maxc * 128);
+    b.lse2 = c.take<float>((size_t)n_heads * 128);
+    b.diag = c.take<float>((size_t)n_heads * b.n_ktiles * 191);
+    b.vert = c.take<float>((size_t)n_heads * n);
+    b.slash = c.take<float>((size_t)n_heads * n);
+    return b;
+}
+
+VsPlanBufs carve_vs_plan(Carver &c, int n, int n_heads, int n_vertical, int n_slash) {
+    VsPlanBufs b{};
+    b.words = n / 32;
+    b.vcap = std::min(n_vertical, n);
+    b.scap = std::min(n_slash, n);
+    const size_t nw = (size_t)n_heads * qtiles(n);
+    b.bits_v = c.take<uint32_t>((size_t)n_heads * b.words);
+    b.bits_s = c.take<uint32_t>((size_t)n_heads * b.words);
+    b.vsorted = c.take<int>((size_t)n_heads * b.vcap);
+    b.nvs = c.take<int>(n_heads);
+    b.soff = c.take<int>((size_t)n_heads * b.scap);
+    b.groups = c.take<int2>((size_t)n_heads * b.scap);
+    b.ngroups = c.take<int>(n_heads);
+    b.nsh = c.take<int>(nw);
+    b.nvert = c.take<int>(nw);
+    b.vlist = c.take<int>(nw * b.vcap);
+    return b;
+}
+
+int bs_head_batch(int n, int n_heads) {
+    const size_t nb = (size_t)n / kBlock;
+    const size_t per = nb * nb * sizeof(float);
+    size_t hb = ((size_t)1 << 30) / std::max<size_t>(per, 1);
+    hb = std::max<size_t>(1, std::min<size_t>(hb, (size_t)n_heads));
+    return (int)hb;
+}
+
+BsEstBufs carve_bs_est(Carver &c, int hkv, int n, int n_heads) {
+    BsEstBufs b{};
+    const size_t nb = (size_t)n / kBlock;
+    b.head_batch = bs_head_batch(n, n_heads);
+    b.qp = c.take<float>((size_t)n_heads * nb * kD);
+    b.kp = c.take<float>((size_t)hkv * nb * kD);
+    b.scores = c.take<float>((size_t)b.head_batch * nb * nb);
+    return b;
+}
+
+struct BsPlanBufs {
+    int *plan, *cnt;
+    int stride;
+};
+
+BsPlanBufs carve_bs_plan(Carver &c, int n, int n_heads, int topk) {
+    BsPlanBufs b{};
+    const int nb = n / kBlock;
+    b.stride = 2 * std::min(topk, nb);
+    const size_t nw = (size_t)n_heads * qtiles(n);
+    b.plan = c.take<int>(nw * b.stride);
+    b.cnt = c.take<int>(nw);
+    return b;
+}
+
+// ------------------------------------------------------------------ devices
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+std::mutex g_dev_mutex;
+int g_dev_ok[64] = {0};  // 0 unknown, 1 sm_100, -1 other
+
+int select_device(const void *ptr) {
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, ptr);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MINF_ERR_CUDA, "cudaPointerGetAttributes: %s", cudaGetErrorString(e));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(MINF_ERR_INVALID, "tensor pointer is not device memory");
+    const int dev = attr.device;
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    std::lock_guard<std::mutex> lk(g_dev_mutex);
+    if (dev >= 0 && dev < 64 && g_dev_ok[dev] == 0) {
+        cudaDeviceProp prop;
+        e = cudaGetDeviceProperties(&prop, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+        g_dev_ok[dev] = prop.major == 10 ? 1 : -1;
+    }
+    if (dev < 0 || dev >= 64 || g_dev_ok[dev] != 1)
+        return fail(MINF_ERR_UNSUPPORTED, "device %d is not an sm_100 (B200-class) GPU", dev);
+    return MINF_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ checks
+struct Common {
+    int hq, hkv, n, n_heads;
+    int ids[MINF_MAX_HEADS];
+};
+
+int check_common(const void *q, const void *k, int hq, int hkv, int n, int d, const int32_t *head_ids,
+                 int n_heads, Common &c) {
+    if (!q || !k) return fail(MINF_ERR_INVALID, "null q or k");
+    if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(MINF_ERR_INVALID, "bad head counts hq=%d hkv=%d", hq, hkv);
+    if (d != kD) return fail(MINF_ERR_UNSUPPORTED, "head dimension %d (only 128)", d);
+    if (n <= 0 || n % kBlock != 0) return fail(MINF_ERR_UNSUPPORTED, "sequence length %d (positive multiple of 64)", n);
+    if (n > (1 << 26)) return fail(MINF_ERR_UNSUPPORTED, "sequence length %d too large", n);
+    if (!aligned16(q) || !aligned16(k)) return fail(MINF_ERR_INVALID, "q/k not 16-byte aligned");
+    if (head_ids) {
+        if (n_heads <= 0 || n_heads > MINF_MAX_HEADS) return fail(MINF_ERR_INVALID, "n_heads=%d", n_heads);
+        for (int i = 0; i < n_heads; ++i) {
+            if (head_ids[i] < 0 || head_ids[i] >= hq) return fail(MINF_ERR_INVALID, "head id %d out of range", head_ids[i]);
+            c.ids[i] = head_ids[i];
+        }
+    } else {
+        if (hq > MINF_MAX_HEADS) return fail(MINF_ERR_INVALID, "hq=%d above %d", hq, MINF_MAX_HEADS);
+        n_heads = hq;
+        for (int i = 0; i < hq; ++i) c.ids[i] = i;
+    }
+    c.hq = hq;
+    c.hkv = hkv;
+    c.n = n;
+    c.n_heads = n_heads;
+    return MINF_OK;
+}
+
+int check_scale(float scale) {
+    if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MINF_ERR_INVALID, "scale must be finite and > 0");
+    return MINF_OK;
+}
+
+int check_ws(void *ws, size_t ws_bytes, size_t need) {
+    if (!ws) return fail(MINF_ERR_INVALID, "null workspace");
+    if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return fail(MINF_ERR_INVALID, "workspace not 256-byte aligned");
+    if (ws_bytes < need) return fail(MINF_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+    return MINF_OK;
+}
+
+// ------------------------------------------------------------------ ops
+size_t bytes_vs_est(int hkv, int n, int n_heads) {
+    Carver c(nullptr, MINF_STATUS_BYTES);
+    carve_vs_est(c, n, n_heads, 1);
+    (void)hkv;
+    return c.off;
+}
+size_t bytes_vs_attn(int n, int n_heads, int nv, int ns) {
+    Carver c(nullptr, MINF_STATUS_BYTES);
+    carve_vs_plan(c, n, n_heads, nv, ns);
+    return c.off;
+}
+size_t bytes_bs_est(int hkv, int n, int n_heads) {
+    Carver c(nullptr, MINF_STATUS_BYTES);
+    carve_bs_est(c, hkv, n, n_heads);
+    return c.off;
+}
+size_t bytes_bs_attn(int n, int n_heads, int topk) {
+    Carver c(nullptr, MINF_STATUS_BYTES);
+    carve_bs_plan(c, n, n_heads, topk);
+    return c.off;
+}
+
+void fill_attn_common(AttnParams &P, const Common &c, float scale, const void *k, const void *v, void *out,
+                      float *lse, void *ws, bool slot_is_id) {
+    P.k = reinterpret_cast<const __nv_bfloat16 *>(k);
+    P.v = reinterpret_cast<const __nv_bfloat16 *>(v);
+    P.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    P.lse = lse;
+    P.hdr = reinterpret_cast<WsHeader *>(ws);
+    P.wait_limit_ns = g_wait_limit_ns.load();
+    P.n = c.n;
+    P.hq = c.hq;
+    P.hkv = c.hkv;
+    P.group = c.hq / c.hkv;
+    P.n_heads = c.n_heads;
+    P.n_qtiles = qtiles(c.n);
+    P.scale_log2 = scale * 1.4426950408889634f;
+    for (int i = 0; i < MINF_MAX_HEADS; ++i) {
+        P.head_ids[i] = i < c.n_heads ? c.ids[i] : 0;
+        P.out_slot[i] = i < c.n_heads ? (slot_is_id ? c.ids[i] : i) : 0;
+    }
+}
+
+cudaError_t encode_attn_maps(AttnParams &P, const void *q, const void *k, const void *v, const Common &c) {
+    cudaError_t e = make_tmap_3d(&P.tmap_q, q, c.hq, c.n);
+    if (e == cudaSuccess) e = make_tmap_3d(&P.tmap_k, k, c.hkv, c.n);
+    if (e == cudaSuccess) e = make_tmap_3d(&P.tmap_v, v, c.hkv, c.n);
+    return e;
+}
+
+int reset_counters(void *ws, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(static_cast<char *>(ws) + offsetof(WsHeader, tiles), 0,
+                                    2 * sizeof(unsigned long long), st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+
+// The bodies below assume checked arguments; `scratch` is the workspace past
+// the status header (or a sub-area of it in the mixed layer).
+int do_vs_estimate(const Common &c, const void *q, const void *k, int last_q, int nv, int ns, float scale,
+                   int32_t *v_idx, int32_t *s_idx, void *ws, char *scratch, cudaStream_t st) {
+    // count the pairs the estimate kernel will form
+    const int group = c.hq / c.hkv;
+    int n_pairs = 0;
+    for (int g = 0; g < c.hkv; ++g) {
+        int cnt = 0;
+        for (int i = 0; i < c.n_heads; ++i) cnt += (c.ids[i] / group == g);
+        n_pairs += (cnt + 1) / 2;
+    }
+    Carver cv(scratch, 0);
+    VsEstBufs b = carve_vs_est(cv, c.n, c.n_heads, n_pairs);
+    VsEstArgs a{};
+    a.q = q;
+    a.k = k;
+    a.hq = c.hq;
+    a.hkv = c.hkv;
+    a.n = c.n;
+    a.last_q = last_q;
+    a.n_heads = c.n_heads;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.head_ids = c.ids;
+    a.n_vertical = nv;
+    a.n_slash = ns;
+    a.v_idx = v_idx;
+    a.s_idx = s_idx;
+    a.hdr = ws;
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    cudaError_t e = run_vs_estimate(a, b, st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "vs_estimate launch");
+}
+
+int do_vs_attention(const Common &c, const void *q, const void *k, const void *v, float scale, const int32_t *v_idx,
+                    int nv, const int32_t *s_idx, int ns, void *out, float *lse, void *ws, char *scratch,
+                    bool slot_is_id, cudaStream_t st) {
+    Carver cv(scratch, 0);
+    VsPlanBufs b = carve_vs_plan(cv, c.n, c.n_heads, nv, ns);
+    cudaError_t e = run_vs_plan(b, v_idx, nv, s_idx, ns, c.n, c.n_heads, qtiles(c.n), st);
+    if (e != cudaSuccess) return cuda_fail(e, "vs plan launch");
+    AttnParams P;
+    memset(&P, 0, sizeof(P));
+    fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
+    e = encode_attn_maps(P, q, k, v, c);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor map");
+    P.vs_groups = b.groups;
+    P.vs_ngroups = b.ngroups;
+    P.vs_gstride = b.scap;
+    P.vs_vert = b.vlist;
+    P.vs_nvert = b.nvert;
+    P.vs_nsh = b.nsh;
+    P.vs_vstride = b.vcap;
+    P.vs_bits_s = b.bits_s;
+    P.vs_bits_v = b.bits_v;
+    P.bit_words = b.words;
+    e = run_attention(PAT_VS, P, st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "vs attention launch");
+}
+
+int do_block_estimate(const Common &c, const void *q, const void *k, int topk, int32_t *blk_idx, int32_t *blk_cnt,
+                      char *scratch, cudaStream_t st) {
+    Carver cv(scratch, 0);
+    BsEstBufs b = carve_bs_est(cv, c.hkv, c.n, c.n_heads);
+    BsEstArgs a{};
+    a.q = q;
+    a.k = k;
+    a.hq = c.hq;
+    a.hkv = c.hkv;
+    a.n = c.n;
+    a.n_heads = c.n_heads;
+    a.topk = topk;
+    a.head_ids = c.ids;
+    a.blk_idx = blk_idx;
+    a.blk_cnt = blk_cnt;
+    cudaError_t e = run_block_estimate(a, b, st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "block_estimate launch");
+}
+
+int do_block_attention(const Common &c, const void *q, const void *k, const void *v, float scale,
+                       const int32_t *blk_idx, const int32_t *blk_cnt, int topk, void *out, float *lse, void *ws,
+                       char *scratch, bool slot_is_id, cudaStream_t st) {
+    Carver cv(scratch, 0);
+    BsPlanBufs b = carve_bs_plan(cv, c.n, c.n_heads, topk);
+    cudaError_t e = run_bs_plan(blk_idx, blk_cnt, topk, c.n_heads, qtiles(c.n), c.n / kBlock, b.plan, b.cnt,
+                                b.stride, st);
+    if (e != cudaSuccess) return cuda_fail(e, "block plan launch");
+    AttnParams P;
+    memset(&P, 0, sizeof(P));
+    fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
+    e = encode_attn_maps(P, q, k, v, c);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor map");
+    P.bs_plan = b.plan;
+    P.bs_cnt = b.cnt;
+    P.bs_stride = b.stride;
+    e = run_attention(PAT_BLOCK, P, st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "block attention launch");
+}
+
+int do_static_attention(int pattern, const Common &c, const void *q, const void *k, const void *v, float scale,
+                        int n_sink, int window, void *out, float *lse, void *ws, bool slot_is_id,
+                        cudaStream_t st) {
+    AttnParams P;
+    memset(&P, 0, sizeof(P));
+    fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
+    cudaError_t e = encode_attn_maps(P, q, k, v, c);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor map");
+    P.n_sink = n_sink;
+    P.window = window;
+    e = run_attention(pattern, P, st);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "attention launch");
+}
+
+}  // namespace
+
+// TMA descriptor of a bf16 [heads][n][128] tensor, box {64, 64, 1}, 128-byte swizzle.
+cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &qres) ==
+                cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)n * kD * 2};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+__global__ void wait_timeout_kernel(WsHeader *hdr, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);  // nothing ever arrives on it
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const WaitCtl wc{&abort_flag, &hdr->status, limit_ns};
+        wait_bounded(smem_u32(&bar), 0, wc);
+    }
+}
+}  // namespace
+
+cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaStream_t st) {
+    wait_timeout_kernel<<<1, 32, 0, st>>>(reinterpret_cast<WsHeader *>(hdr), limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace minf
+
+using namespace minf;
+
+extern "C" {
+
+size_t minf_workspace_bytes(int op, int hq, int hkv, int n, int n_heads, int p1, int p2, int p3) {
+    if (hq <= 0 || hkv <= 0 || hq % hkv || n <= 0 || n % kBlock) return 0;
+    if (n_heads <= 0) n_heads = hq;
+    switch (op) {
+    case MINF_OP_VS_ESTIMATE:
+        return bytes_vs_est(hkv, n, n_heads);
+    case MINF_OP_VS_ATTENTION:
+        if (p1 < 1 || p2 < 1) return 0;
+        return bytes_vs_attn(n, n_heads, p1, p2);
+    case MINF_OP_BLOCK_ESTIMATE:
+        return bytes_bs_est(hkv, n, n_heads);
+    case MINF_OP_BLOCK_ATTENTION:
+        if (p1 < 1) return 0;
+        return bytes_bs_attn(n, n_heads, p1);
+    case MINF_OP_ASHAPE_ATTENTION:
+    case MINF_OP_DENSE_ATTENTION:
+        return MINF_STATUS_BYTES;
+    case MINF_OP_MIXED_LAYER: {
+        if (p1 < 1 || p2 < 1 || p3 < 1) return 0;
+        const int nb = n / kBlock;
+        Carver c(nullptr, MINF_STATUS_BYTES);
+        c.take<int>((size_t)hq * p1);
+        c.take<int>((size_t)hq * p2);
+        c.take<int>((size_t)hq * nb * p3);
+        c.take<int>((size_t)hq * nb);
+        const size_t sub = std::max(std::max(bytes_vs_est(hkv, n, hq), bytes_vs_attn(n, hq, p1, p2)),
+                                    std::max(bytes_bs_est(hkv, n, hq), bytes_bs_attn(n, hq, p3)));
+        c.take<char>(sub);
+        return c.off;
+    }
+    }
+    return 0;
+}
+
+int minf_vs_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d, int last_q,
+                     int n_vertical, int n_slash, float scale, const int32_t *head_ids, int n_heads,
+                     int32_t *v_idx, int32_t *s_idx, void *ws, size_t ws_bytes, minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v_idx || !s_idx) return fail(MINF_ERR_INVALID, "null v_idx or s_idx");
+    if (n_vertical < 1 || n_slash < 1) return fail(MINF_ERR_INVALID, "budgets must be >= 1");
+    if (last_q < 1) return fail(MINF_ERR_INVALID, "last_q must be >= 1");
+    if (last_q > 64) return fail(MINF_ERR_UNSUPPORTED, "last_q %d above 64", last_q);
+    if ((rc = check_ws(ws, ws_bytes, bytes_vs_est(hkv, n, c.n_heads)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    return do_vs_estimate(c, q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws,
+                          static_cast<char *>(ws) + MINF_STATUS_BYTES, (cudaStream_t)stream);
+}
+
+int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                      float scale, const int32_t *head_ids, int n_heads, const int32_t *v_idx, int n_vertical,
+                      const int32_t *s_idx, int n_slash, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                      minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out || !v_idx || !s_idx) return fail(MINF_ERR_INVALID, "null v, out or index rows");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if (n_vertical < 1 || n_slash < 1) return fail(MINF_ERR_INVALID, "budgets must be >= 1");
+    if ((rc = check_ws(ws, ws_bytes, bytes_vs_attn(n, c.n_heads, n_vertical, n_slash)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
+    return do_vs_attention(c, q, k, v, scale, v_idx, n_vertical, s_idx, n_slash, out, lse, ws,
+                           static_cast<char *>(ws) + MINF_STATUS_BYTES, false, (cudaStream_t)stream);
+}
+
+int minf_block_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d, int block, int topk,
+                        const int32_t *head_ids, int n_heads, int32_t *blk_idx, int32_t *blk_cnt, void *ws,
+                        size_t ws_bytes, minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if (block != kBlock) return fail(MINF_ERR_UNSUPPORTED, "block %d (only 64)", block);
+    if (!blk_idx || !blk_cnt) return fail(MINF_ERR_INVALID, "null blk_idx or blk_cnt");
+    if (topk < 1) return fail(MINF_ERR_INVALID, "topk must be >= 1");
+    if (n / kBlock > 32768) return fail(MINF_ERR_UNSUPPORTED, "more than 32768 blocks");
+    if ((rc = check_ws(ws, ws_bytes, bytes_bs_est(hkv, n, c.n_heads)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    return do_block_estimate(c, q, k, topk, blk_idx, blk_cnt, static_cast<char *>(ws) + MINF_STATUS_BYTES,
+                             (cudaStream_t)stream);
+}
+
+int minf_block_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                         float scale, const int32_t *head_ids, int n_heads, const int32_t *blk_idx,
+                         const int32_t *blk_cnt, int topk, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                         minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out || !blk_idx || !blk_cnt) return fail(MINF_ERR_INVALID, "null v, out or block rows");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if (topk < 1) return fail(MINF_ERR_INVALID, "topk must be >= 1");
+    if ((rc = check_ws(ws, ws_bytes, bytes_bs_attn(n, c.n_heads, topk)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
+    return do_block_attention(c, q, k, v, scale, blk_idx, blk_cnt, topk, out, lse, ws,
+                              static_cast<char *>(ws) + MINF_STATUS_BYTES, false, (cudaStream_t)stream);
+}
+
+int minf_ashape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                          float scale, const int32_t *head_ids, int n_heads, int n_sink, int window, minf_bf16 *out,
+                          float *lse, void *ws, size_t ws_bytes, minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out) return fail(MINF_ERR_INVALID, "null v or out");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if (n_sink < 0 || window < 1) return fail(MINF_ERR_INVALID, "n_sink >= 0 and window >= 1 required");
+    if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
+    if ((rc = select_device(q))) return rc;
+    if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
+    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, out, lse, ws, false,
+                               (cudaStream_t)stream);
+}
+
+int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                         float scale, const int32_t *head_ids, int n_heads, minf_bf16 *out, float *lse, void *ws,
+                         size_t ws_bytes, minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out) return fail(MINF_ERR_INVALID, "null v or out");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
+    if ((rc = select_device(q))) return rc;
+    if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
+    return do_static_attention(PAT_DENSE, c, q, k, v, scale, 0, 1, out, lse, ws, false, (cudaStream_t)stream);
+}
+
+int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                     float scale, const int8_t *head_pattern, int last_q, int n_vertical, int n_slash, int topk,
+                     int n_sink, int window, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                     minf_stream_t stream) {
+    Common all;
+    int rc = check_common(q, k, hq, hkv, n, d, nullptr, hq, all);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out || !head_pattern) return fail(MINF_ERR_INVALID, "null v, out or head_pattern");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if (n_vertical < 1 || n_slash < 1 || topk < 1 || last_q < 1 || n_sink < 0 || window < 1)
+        return fail(MINF_ERR_INVALID, "bad pattern parameters");
+    if (last_q > 64) return fail(MINF_ERR_UNSUPPORTED, "last_q %d above 64", last_q);
+    if (n / kBlock > 32768) return fail(MINF_ERR_UNSUPPORTED, "more than 32768 blocks");
+    Common sub[4];
+    for (int p = 0; p < 4; ++p) {
+        sub[p] = all;
+        sub[p].n_heads = 0;
+    }
+    for (int h = 0; h < hq; ++h) {
+        const int p = head_pattern[h];
+        if (p < 0 || p > 3) return fail(MINF_ERR_INVALID, "head %d: pattern code %d", h, p);
+        sub[p].ids[sub[p].n_heads++] = h;
+    }
+    const size_t need = minf_workspace_bytes(MINF_OP_MIXED_LAYER, hq, hkv, n, hq, n_vertical, n_slash, topk);
+    if ((rc = check_ws(ws, ws_bytes, need))) return rc;
+    if ((rc = select_device(q))) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = reset_counters(ws, st))) return rc;
+    const int nb = n / kBlock;
+    Carver c(ws, MINF_STATUS_BYTES);
+    int32_t *v_idx = c.take<int32_t>((size_t)hq * n_vertical);
+    int32_t *s_idx = c.take<int32_t>((size_t)hq * n_slash);
+    int32_t *blk_idx = c.take<int32_t>((size_t)hq * nb * topk);
+    int32_t *blk_cnt = c.take<int32_t>((size_t)hq * nb);
+    char *scratch = c.take<char>(0);
+    // estimates first (VS, then Block-Sparse), then the attention of every group
+    if (sub[PAT_VS].n_heads) {
+        rc = do_vs_estimate(sub[PAT_VS], q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws, scratch, st);
+        if (rc) return rc;
+        rc = do_vs_attention(sub[PAT_VS], q, k, v, scale, v_idx, n_vertical, s_idx, n_slash, out, lse, ws, scratch,
+                             true, st);
+        if (rc) return rc;
+    }
+    if (sub[PAT_BLOCK].n_heads) {
+        rc = do_block_estimate(sub[PAT_BLOCK], q, k, topk, blk_idx, blk_cnt, scratch, st);
+        if (rc) return rc;
+        rc = do_block_attention(sub[PAT_BLOCK], q, k, v, scale, blk_idx, blk_cnt, topk, out, lse, ws, scratch, true,
+                                st);
+        if (rc) return rc;
+    }
+    if (sub[PAT_ASHAPE].n_heads) {
+        rc = do_static_attention(PAT_ASHAPE, sub[PAT_ASHAPE], q, k, v, scale, n_sink, window, out, lse, ws, true, st);
+        if (rc) return rc;
+    }
+    if (sub[PAT_DENSE].n_heads) {
+        rc = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, out, lse, ws, true, st);
+        if (rc) return rc;
+    }
+    return MINF_OK;
+}
+
+int minf_status(void *ws, minf_stream_t stream) {
+    if (!ws) return fail(MINF_ERR_INVALID, "null workspace");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int status = 0;
+    e = cudaMemcpy(&status, ws, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy status");
+    if (status != 0) {
+        e = cudaMemset(ws, 0, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset status");
+    }
+    return status;
+}
+
+int minf_stats(void *ws, minf_stream_t stream, uint64_t *tiles, uint64_t *pairs) {
+    if (!ws || !tiles || !pairs) return fail(MINF_ERR_INVALID, "null argument");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    WsHeader h;
+    e = cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy stats");
+    *tiles = h.tiles;
+    *pairs = h.pairs;
+    return MINF_OK;
+}
+
+void minf_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 2000000000ull); }
+
+int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_stream_t stream) {
+    int rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES);
+    if (rc) return rc;
+    if ((rc = select_device(ws))) return rc;
+    cudaError_t e = run_wait_timeout_check(ws, limit_ns, (cudaStream_t)stream);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "wait check launch");
+}
+
+const char *minf_version(void) { return "minf-b200 0.1.0 (sm_100a)"; }
+
+const char *minf_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

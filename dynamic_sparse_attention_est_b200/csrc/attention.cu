@@ -1,0 +1,730 @@
+// attention.cu -- causal sparse FlashAttention on sm_100a (tcgen05 + TMEM + TMA).
+//
+// One CTA computes one work item: 128 query rows of one q-head against the key
+// tiles its pattern selects.  A key tile is 128 keys made of two 64-key halves;
+// each half is a contiguous key range loaded by TMA or a list of gathered keys
+// (vertical lines), so every tile is one dense M=128, N=128 contraction on the
+// tensor cores whatever the pattern (the index-shifting idea of the AICon talk
+// "以 KV 缓存为中心的高效长文本方法": turn verticals and slashes into dense blocks;
+// news article "单卡A100实现百万token推理…", Figure 4: slashes as dense blocks,
+// verticals as 1x64 pieces).  The pattern's exact mask is applied per element
+// inside each tile, so the result is the token-exact masked softmax.
+//
+// Warp roles (256 threads):
+//   warp 0      TMA producer for Q and K (+ cp.async gathers of vertical keys)
+//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
+//   warp 2      TMA producer for V (+ gathers)
+//   warp 3      idle
+//   warps 4..7  softmax warpgroup: thread r owns query row r (TMEM lane r)
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+// S = Q K^T (SS MMA), P = exp(S - m) as bf16 written back to TMEM, O += P V with
+// P read from TMEM (TS MMA).  Online softmax in fp32 with lazy rescaling: the
+// running max only moves when a row's max grows by more than 2^8.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace minf {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 bf16
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kSmemQ + kTileBytes;
+constexpr uint32_t kSmemV = kSmemK + 2 * kTileBytes;
+constexpr uint32_t kSmemBar = kSmemV + 2 * kTileBytes;
+constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
+
+enum : int {
+    B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 3, B_V_FULL = 5, B_V_EMPTY = 7,
+    B_S_FULL = 9, B_P_FULL = 11, B_O_DONE = 13, B_ALL_DONE = 14, B_COUNT = 15
+};
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, true);
+
+// ------------------------------------------------------------------ tile plans
+// Every role walks the same deterministic sequence of half-tiles.
+template <int PAT>
+struct TileGen {
+    int r0, rmax, total, emitted;
+    // A-shape
+    int sink_h, w_lo, split;
+    // Block-Sparse
+    const int *plan;
+    // Vertical-Slash
+    const int2 *groups;
+    int ng, gi, cur_a, cur_b, nsh, nvert;
+
+    __device__ void init(const AttnParams &P, int hp, int t) {
+        r0 = t * kTileM;
+        rmax = min(r0 + kTileM - 1, P.n - 1);
+        emitted = 0;
+        const int nb64 = P.n / kHalf;
+        const int hi = min(2 * t + 1, nb64 - 1);
+        if constexpr (PAT == PAT_DENSE) {
+            total = hi + 1;
+        } else if constexpr (PAT == PAT_ASHAPE) {
+            sink_h = min((P.n_sink + kHalf - 1) / kHalf, nb64);
+            w_lo = max(0, r0 - P.window + 1) / kHalf;
+            split = w_lo > sink_h;
+            total = split ? sink_h + (hi - w_lo + 1) : hi + 1;
+        } else if constexpr (PAT == PAT_BLOCK) {
+            const int w = hp * P.n_qtiles + t;
+            plan = P.bs_plan + (size_t)w * P.bs_stride;
+            total = P.bs_cnt[w];
+        } else {
+            const int w = hp * P.n_qtiles + t;
+            groups = P.vs_groups + (size_t)hp * P.vs_gstride;
+            ng = P.vs_ngroups[hp];
+            gi = 0;
+            cur_a = 1;
+            cur_b = 0;
+            nsh = P.vs_nsh[w];
+            nvert = P.vs_nvert[w];
+            total = nsh + (nvert + kHalf - 1) / kHalf;
+        }
+    }
+
+    __device__ int tiles() const { return (total + 1) >> 1; }
+
+    __device__ HalfDesc next(const AttnParams &P) {
+        HalfDesc h{HALF_EMPTY, 0, 0, 0};
+        if (emitted >= total) {
+            ++emitted;
+            return h;
+        }
+        const int i = emitted++;
+        if constexpr (PAT == PAT_DENSE) {
+            h.kind = HALF_RANGE;
+            h.ks = i * kHalf;
+            h.len = kHalf;
+            h.flags = HF_ROWS0 | HF_ROWS1 | (h.ks + kHalf - 1 <= r0 ? HF_FULL : 0);
+        } else if constexpr (PAT == PAT_ASHAPE) {
+            const int blk = (!split || i < sink_h) ? i : w_lo + (i - sink_h);
+            h.kind = HALF_RANGE;
+            h.ks = blk * kHalf;
+            h.len = kHalf;
+            const bool full = (h.ks + kHalf - 1 <= r0) &&
+                              (h.ks + kHalf - 1 < P.n_sink || (r0 + kTileM - 1) - h.ks < P.window);
+            h.flags = HF_ROWS0 | HF_ROWS1 | (full ? HF_FULL : 0);
+        } else if constexpr (PAT == PAT_BLOCK) {
+            const int e = __ldg(plan + i);
+            const int rows = e & 3;
+            h.kind = HALF_RANGE;
+            h.ks = (e >> 2) * kHalf;
+            h.len = kHalf;
+            h.flags = (rows << 1) | ((rows == 3 && h.ks + kHalf - 1 <= r0) ? HF_FULL : 0);
+        } else {
+            if (i < nsh) {
+                if (cur_a > cur_b) {
+                    while (gi < ng) {
+                        const int2 g = __ldg(groups + gi);
+                        ++gi;
+                        const int a = max(0, r0 - g.y);
+                        const int b = min(r0 + kTileM - 1 - g.x, rmax);
+                        if (b >= a) {
+                            cur_a = a;
+                            cur_b = b;
+                            break;
+                        }
+                    }
+                }
+                if (cur_a <= cur_b) {
+                    h.kind = HALF_RANGE;
+                    h.ks = cur_a;
+                    h.len = min(kHalf, cur_b - cur_a + 1);
+                    h.flags = HF_ROWS0 | HF_ROWS1;
+                    cur_a += kHalf;
+                }
+            } else {
+                const int m = i - nsh;
+                h.kind = HALF_GATHER;
+                h.ks = m * kHalf;
+                h.len = min(kHalf, nvert - m * kHalf);
+                h.flags = HF_ROWS0 | HF_ROWS1;
+            }
+        }
+        return h;
+    }
+};
+
+// Element mask of one half for query row q (= r0 + r): bit c set iff key c of
+// the half is inside the pattern's mask for q.
+template <int PAT>
+__device__ __forceinline__ uint64_t half_mask(const AttnParams &P, const HalfDesc &h, int q, int r,
+                                              const int *vlist, const uint32_t *bits_s,
+                                              const uint32_t *bits_v) {
+    if (h.kind == HALF_EMPTY) return 0ull;
+    if (h.flags & HF_FULL) return ~0ull;
+    const uint64_t causal = low_bits(q - h.ks + 1);
+    if constexpr (PAT == PAT_DENSE) {
+        return causal;
+    } else if constexpr (PAT == PAT_ASHAPE) {
+        const uint64_t sink = low_bits(P.n_sink - h.ks);
+        const int c0 = q - h.ks - P.window + 1;  // first column inside the window
+        const uint64_t win = c0 <= 0 ? ~0ull : (c0 >= 64 ? 0ull : (~0ull << c0));
+        return causal & (sink | win);
+    } else if constexpr (PAT == PAT_BLOCK) {
+        const int half_row = r >> 6;
+        return (h.flags & (HF_ROWS0 << half_row)) ? causal : 0ull;
+    } else {
+        const uint64_t lenm = low_bits(h.len);
+        if (h.kind == HALF_RANGE) {
+            // slash: offset q - (ks + c) in S; vertical: key ks + c in V
+            const uint64_t ws = bits64_at(bits_s, P.bit_words, q - h.ks - 63);
+            const uint64_t wv = bits64_at(bits_v, P.bit_words, h.ks);
+            return causal & lenm & (__brevll(ws) | wv);
+        }
+        // gathered verticals, ascending: keep those <= q
+        const int *lst = vlist + h.ks;
+        int lo = 0, hi = h.len;  // first index with key > q
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(lst + mid) <= q) lo = mid + 1;
+            else hi = mid;
+        }
+        return low_bits(lo) & lenm;
+    }
+}
+
+// Loads the two halves of one K or V tile into a 128-row, 128B-swizzled stage.
+template <int PAT>
+__device__ __forceinline__ void load_tile(uint32_t stage, uint32_t bar, const HalfDesc (&hd)[2],
+                                          const CUtensorMap *map, const __nv_bfloat16 *raw,
+                                          int g, int n, const int *vlist, int lane) {
+    uint32_t tma_bytes = 0;
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+        if (hd[s].kind != HALF_GATHER) tma_bytes += 2 * 8192;
+    if (lane == 0) {
+        mbar_expect_tx(bar, tma_bytes);
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (hd[s].kind == HALF_GATHER) continue;
+            const int ks = hd[s].kind == HALF_RANGE ? hd[s].ks : 0;
+            tma_load_3d(stage + s * 8192, map, bar, 0, ks, g);
+            tma_load_3d(stage + 16384 + s * 8192, map, bar, 64, ks, g);
+        }
+    }
+    bool gathered = false;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        if (hd[s].kind != HALF_GATHER) continue;
+        gathered = true;
+        const int *lst = vlist + hd[s].ks;
+        for (int rr = lane; rr < kHalf; rr += 32) {
+            const int key = __ldg(lst + min(rr, hd[s].len - 1));
+            const __nv_bfloat16 *src = raw + ((size_t)g * n + key) * kD;
+            const int row = s * kHalf + rr;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const uint32_t dst = stage + (u >> 3) * 16384 + row * 128 + (((u & 7) ^ (row & 7)) << 4);
+                cp_async16(dst, src + u * 8);
+            }
+        }
+    }
+    if (gathered) {
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
+template <int PAT>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + kSmemQ, sK = sbase + kSmemK, sV = sbase + kSmemV;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + B_COUNT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT + 1);
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = P.n_qtiles - 1 - (int)(blockIdx.x / P.n_heads);  // heaviest tiles first
+    const int hp = (int)(blockIdx.x % P.n_heads);
+    const int h = P.head_ids[hp];
+    const int g = h / P.group;
+    const int w_item = hp * P.n_qtiles + t;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_Q_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_K_FULL + s), 1);
+            mbar_init(bar(B_K_EMPTY + s), 1);
+            mbar_init(bar(B_V_FULL + s), 1);
+            mbar_init(bar(B_V_EMPTY + s), 1);
+            mbar_init(bar(B_S_FULL + s), 1);
+            mbar_init(bar(B_P_FULL + s), 128);
+        }
+        mbar_init(bar(B_O_DONE), 1);
+        mbar_init(bar(B_ALL_DONE), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&P.tmap_q);
+        tma_prefetch_desc(&P.tmap_k);
+        tma_prefetch_desc(&P.tmap_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl wc{abort_flag, P.hdr ? &P.hdr->status : nullptr, P.wait_limit_ns};
+
+    TileGen<PAT> gen;
+    gen.init(P, hp, t);
+    const int T = gen.tiles();
+    const int *vlist = nullptr;
+    if constexpr (PAT == PAT_VS) vlist = P.vs_vert + (size_t)w_item * P.vs_vstride;
+
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------ producers
+        const bool is_k = warp == 0;
+        const CUtensorMap *map = is_k ? &P.tmap_k : &P.tmap_v;
+        const __nv_bfloat16 *raw = is_k ? P.k : P.v;
+        const uint32_t stage0 = is_k ? sK : sV;
+        const int full0 = is_k ? B_K_FULL : B_V_FULL, empty0 = is_k ? B_K_EMPTY : B_V_EMPTY;
+        if (is_k && lane == 0 && T > 0) {
+            const int r0 = t * kTileM;
+            mbar_expect_tx(bar(B_Q_FULL), 4 * 8192);
+            tma_load_3d(sQ, &P.tmap_q, bar(B_Q_FULL), 0, r0, h);
+            tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q_FULL), 64, r0, h);
+            tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q_FULL), 0, r0 + 64, h);
+            tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q_FULL), 64, r0 + 64, h);
+            mbar_arrive(bar(B_Q_FULL));
+        }
+        int issued = 0;
+        for (int j = 0; j < T; ++j) {
+            const int s = j & 1;
+            const uint32_t ph = (j >> 1) & 1;
+            HalfDesc hd[2];
+            hd[0] = gen.next(P);
+            hd[1] = gen.next(P);
+            if (!wait_bounded(bar(empty0 + s), ph ^ 1, wc)) break;
+            load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
+            issued = j + 1;
+        }
+        if (*abort_flag && lane == 0) {
+            // drain: let the loads already issued land before the CTA exits
+            WaitCtl drain{abort_flag, nullptr, 50000000ull};
+            volatile int no_abort = 0;
+            drain.abort_flag = &no_abort;
+            for (int j = max(0, issued - 2); j < issued; ++j)
+                wait_bounded(bar(full0 + (j & 1)), (j >> 1) & 1, drain);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && T > 0) {
+            const uint32_t tS[2] = {tmem + 0, tmem + 128};
+            const uint32_t tO = tmem + 256;
+            const uint32_t tP[2] = {tmem + 384, tmem + 448};
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!wait_bounded(bar(B_K_FULL + s), (j >> 1) & 1, wc)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tS[s], sdesc_sw128(sQ + off, 16, 1024),
+                            sdesc_sw128(sK + s * kTileBytes + off, 16, 1024), kIdescQK, kk != 0);
+                }
+                umma_commit(bar(B_K_EMPTY + s));
+                umma_commit(bar(B_S_FULL + s));
+                return true;
+            };
+            bool ok = wait_bounded(bar(B_Q_FULL), 0, wc);
+            if (ok) {
+                tc_fence_after();
+                ok = issue_s(0);
+                if (ok && T > 1) ok = issue_s(1);
+            }
+            for (int j = 0; ok && j < T; ++j) {
+                const int b = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!wait_bounded(bar(B_P_FULL + b), ph, wc)) break;
+                if (!wait_bounded(bar(B_V_FULL + b), ph, wc)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tO, tP[b] + kk * 8, sdesc_sw128(sV + b * kTileBytes + kk * 2048, 16384, 1024),
+                            kIdescPV, (j | kk) != 0);
+                umma_commit(bar(B_V_EMPTY + b));
+                umma_commit(bar(B_O_DONE));
+                if (j + 2 < T && !issue_s(j + 2)) break;
+            }
+            // always close: the epilogue (or the abort path) waits for this
+            umma_commit(bar(B_ALL_DONE));
+            if (P.hdr) atomicAdd(&P.hdr->tiles, (unsigned long long)T);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax
+        const int r = threadIdx.x - 128;
+        const int q = t * kTileM + r;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS[2] = {tmem + lane_off + 0, tmem + lane_off + 128};
+        const uint32_t tO = tmem + lane_off + 256;
+        const uint32_t tP[2] = {tmem + lane_off + 384, tmem + lane_off + 448};
+        const float sl2 = P.scale_log2;
+        const uint32_t *bits_s = nullptr, *bits_v = nullptr;
+        if constexpr (PAT == PAT_VS) {
+            bits_s = P.vs_bits_s + (size_t)hp * P.bit_words;
+            bits_v = P.vs_bits_v + (size_t)hp * P.bit_words;
+        }
+        float m_run = -INFINITY, l_run = 0.f;
+        unsigned long long pairs = 0;
+        bool ok = true;
+        for (int j = 0; j < T && ok; ++j) {
+            const int b = j & 1;
+            const uint32_t ph = (j >> 1) & 1;
+            HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
+            const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, bits_s, bits_v);
+            const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, bits_s, bits_v);
+            if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
+            if (!wait_bounded(bar(B_S_FULL + b), ph, wc)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS[b] + c * 32, sr[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint64_t mk = c < 2 ? mk0 : mk1;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int bit = (c & 1) * 32 + e;
+                    float x = __uint_as_float(sr[c][e]);
+                    x = ((mk >> bit) & 1ull) ? x : -INFINITY;
+                    sr[c][e] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+            }
+            mx *= sl2;
+            const float m_new = fmaxf(m_run, mx);
+            if (m_new > m_run + 8.0f) {
+                const float alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
+                if (j > 0 && m_run != -INFINITY) {
+                    // O holds tiles < j: wait for P(j-1) V(j-1), then rescale it in TMEM
+                    if (!wait_bounded(bar(B_O_DONE), (j - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_ld_wait(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tO + c * 32, o);
+                    }
+                }
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            const float m_use = m_run == -INFINITY ? 0.f : m_run;
+            float lsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_use));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_use));
+                    lsum += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                // reuse the first 16 registers of sr[c] as the packed row chunk
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sr[c][e] = pk[e];
+            }
+            l_run += lsum;
+            uint32_t pp[2][32];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                pp[0][e] = sr[0][e];
+                pp[0][16 + e] = sr[1][e];
+                pp[1][e] = sr[2][e];
+                pp[1][16 + e] = sr[3][e];
+            }
+            tmem_st32(tP[b], pp[0]);
+            tmem_st32(tP[b] + 32, pp[1]);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(B_P_FULL + b));
+        }
+        // epilogue
+        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            const size_t orow = (size_t)P.out_slot[hp] * P.n + min(q, P.n - 1);
+            uint4 *dst = reinterpret_cast<uint4 *>(P.out + orow * kD);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                if (T > 0) {  // uniform over the CTA: every lane of the warp loads
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait(o);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                if (q < P.n) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                            __uint_as_float(o[2 * e + 1]) * inv_l);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            if (q < P.n && P.lse)
+                P.lse[orow] =
+                    l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        }
+        if (P.hdr) {
+#pragma unroll
+            for (int s = 16; s > 0; s >>= 1) pairs += __shfl_xor_sync(0xffffffffu, pairs, s);
+            if (lane == 0) atomicAdd(&P.hdr->pairs, pairs);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ planners
+// Block-Sparse: per work item (two 64-row query blocks), merge the two
+// ascending block lists into one list of half entries (block << 2 | rows).
+__global__ void bs_plan_kernel(const int *blk_idx, const int *blk_cnt, int topk, int n_heads,
+                               int n_qtiles, int nb, int *plan, int *cnt, int stride) {
+    const int w = blockIdx.x * blockDim.x + threadIdx.x;
+    if (w >= n_heads * n_qtiles) return;
+    const int hp = w / n_qtiles, t = w % n_qtiles;
+    const int b0 = 2 * t, b1 = 2 * t + 1;
+    const int *l0 = blk_idx + ((size_t)hp * nb + b0) * topk;
+    const int *l1 = b1 < nb ? blk_idx + ((size_t)hp * nb + b1) * topk : nullptr;
+    const int c0 = min(max(blk_cnt[(size_t)hp * nb + b0], 0), topk);
+    const int c1 = l1 ? min(max(blk_cnt[(size_t)hp * nb + b1], 0), topk) : 0;
+    int i0 = 0, i1 = 0, last0 = -1, last1 = -1, out = 0;
+    int *dst = plan + (size_t)w * stride;
+    // entries that are negative, in the future of their block, or not above the
+    // previous entry of their list are skipped
+    auto next0 = [&]() -> int {
+        while (i0 < c0) {
+            const int j = l0[i0];
+            if (j > last0 && j >= 0 && j <= b0) return j;
+            ++i0;
+        }
+        return INT_MAX;
+    };
+    auto next1 = [&]() -> int {
+        while (i1 < c1) {
+            const int j = l1[i1];
+            if (j > last1 && j >= 0 && j <= b1) return j;
+            ++i1;
+        }
+        return INT_MAX;
+    };
+    for (;;) {
+        const int j0 = next0(), j1 = next1();
+        if (j0 == INT_MAX && j1 == INT_MAX) break;
+        const int j = min(j0, j1);
+        int rows = 0;
+        if (j0 == j) { rows |= 1; last0 = j; ++i0; }
+        if (j1 == j) { rows |= 2; last1 = j; ++i1; }
+        dst[out++] = (j << 2) | rows;
+    }
+    cnt[w] = out;
+}
+
+// Vertical-Slash: mark the index rows into per-head bitmaps (order-free,
+// duplicates merge, out-of-range entries ignored).
+__global__ void vs_mark_kernel(const int *v_idx, int n_vertical, const int *s_idx, int n_slash, int n,
+                               uint32_t *bits_v, uint32_t *bits_s, int words) {
+    const int hp = blockIdx.x;
+    for (int i = threadIdx.x; i < n_vertical; i += blockDim.x) {
+        const int x = v_idx[(size_t)hp * n_vertical + i];
+        if (x >= 0 && x < n) atomicOr(bits_v + (size_t)hp * words + (x >> 5), 1u << (x & 31));
+    }
+    for (int i = threadIdx.x; i < n_slash; i += blockDim.x) {
+        const int x = s_idx[(size_t)hp * n_slash + i];
+        if (x >= 0 && x < n) atomicOr(bits_s + (size_t)hp * words + (x >> 5), 1u << (x & 31));
+    }
+}
+
+// Ordered extraction of the set bits of a bitmap by one warp.
+__device__ int warp_extract_bits(const uint32_t *bm, int words, int *out, int cap, int lane) {
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        uint32_t word = (w0 + lane < words) ? bm[w0 + lane] : 0u;
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, s);
+            if (lane >= s) incl += y;
+        }
+        int pos = base + incl - c;
+        while (word) {
+            const int b = __ffs(word) - 1;
+            if (pos < cap) out[pos] = (w0 + lane) * 32 + b;
+            ++pos;
+            word &= word - 1;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return min(base, cap);
+}
+
+// Per head: sorted distinct verticals, and slash offsets merged into groups
+// whose 128-row key ranges touch (consecutive offsets at most 128 apart).
+__global__ void vs_extract_kernel(const uint32_t *bits_v, const uint32_t *bits_s, int words, int *vsorted,
+                                  int *nvs, int vcap, int *soff, int scap, int2 *groups, int *ngroups) {
+    const int hp = blockIdx.x, lane = threadIdx.x;
+    const int cv = warp_extract_bits(bits_v + (size_t)hp * words, words, vsorted + (size_t)hp * vcap, vcap, lane);
+    const int cs = warp_extract_bits(bits_s + (size_t)hp * words, words, soff + (size_t)hp * scap, scap, lane);
+    __syncwarp();
+    const int *so = soff + (size_t)hp * scap;
+    int2 *gr = groups + (size_t)hp * scap;
+    int ng = 0;
+    for (int e0 = 0; e0 < cs; e0 += 32) {
+        const int e = e0 + lane;
+        bool start = false;
+        if (e < cs) start = (e == 0) || (so[e] - so[e - 1] > kTileM);
+        const uint32_t bal = __ballot_sync(0xffffffffu, start);
+        if (start) gr[ng + __popc(bal & ((1u << lane) - 1u))].x = e;
+        ng += __popc(bal);
+    }
+    __syncwarp();
+    for (int g0 = 0; g0 < ng; g0 += 32) {
+        const int gg = g0 + lane;
+        int s = gg < ng ? gr[gg].x : cs;
+        int nxt = __shfl_down_sync(0xffffffffu, s, 1);
+        if (lane == 31) nxt = (g0 + 32 < ng) ? gr[g0 + 32].x : cs;
+        if (gg >= ng - 1) nxt = cs;
+        __syncwarp();
+        if (gg < ng) gr[gg] = make_int2(so[s], so[nxt - 1]);
+        __syncwarp();
+    }
+    if (lane == 0) {
+        nvs[hp] = cv;
+        ngroups[hp] = ng;
+    }
+}
+
+__device__ __forceinline__ bool any_bits(const uint32_t *bm, int lo, int hi) {
+    for (int w = lo >> 5; w <= (hi >> 5); ++w) {
+        uint32_t m = 0xffffffffu;
+        if (w == (lo >> 5)) m &= 0xffffffffu << (lo & 31);
+        if (w == (hi >> 5)) m &= 0xffffffffu >> (31 - (hi & 31));
+        if (bm[w] & m) return true;
+    }
+    return false;
+}
+
+// Per work item (one warp): number of slash half-tiles, and the ascending list
+// of vertical keys that no slash range of this 128-row tile covers.
+__global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap, const int2 *groups,
+                                   const int *ngroups, int gstride, const uint32_t *bits_s, int words, int n,
+                                   int n_heads, int n_qtiles, int *nsh, int *nvert, int *vlist) {
+    const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= n_heads * n_qtiles) return;
+    const int hp = w / n_qtiles, t = w % n_qtiles;
+    const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, n - 1);
+    const int2 *gr = groups + (size_t)hp * gstride;
+    const int ng = ngroups[hp];
+    int halves = 0;
+    for (int i = lane; i < ng; i += 32) {
+        const int2 gg = gr[i];
+        const int a = max(0, r0 - gg.y), b = min(r0 + kTileM - 1 - gg.x, rmax);
+        if (b >= a) halves += (b - a + kHalf) / kHalf;
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, s);
+    const int *vs = vsorted + (size_t)hp * vcap;
+    const uint32_t *bs = bits_s + (size_t)hp * words;
+    int *dst = vlist + (size_t)w * vcap;
+    const int cv = nvs[hp];
+    int out = 0;
+    for (int e0 = 0; e0 < cv; e0 += 32) {
+        const int e = e0 + lane;
+        bool keep = false;
+        if (e < cv) {
+            const int x = vs[e];
+            if (x <= rmax) {
+                const int lo = max(0, r0 - x), hi = min(r0 + kTileM - 1 - x, n - 1);
+                keep = !any_bits(bs, lo, hi);
+            }
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) dst[out + __popc(bal & ((1u << lane) - 1u))] = vs[e];
+        out += __popc(bal);
+    }
+    if (lane == 0) {
+        nsh[w] = halves;
+        nvert[w] = out;
+    }
+}
+
+template <int PAT>
+cudaError_t launch_attn(const AttnParams &P, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<PAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = P.n_heads * P.n_qtiles;
+    if (grid == 0) return cudaSuccess;
+    attn_kernel<PAT><<<grid, kThreads, kSmemBytes, st>>>(P);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st) {
+    switch (pattern) {
+    case PAT_DENSE: return launch_attn<PAT_DENSE>(P, st);
+    case PAT_ASHAPE: return launch_attn<PAT_ASHAPE>(P, st);
+    case PAT_BLOCK: return launch_attn<PAT_BLOCK>(P, st);
+    case PAT_VS: return launch_attn<PAT_VS>(P, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_heads, int n_qtiles, int nb,
+                        int *plan, int *cnt, int stride, cudaStream_t st) {
+    const int nw = n_heads * n_qtiles;
+    bs_plan_kernel<<<(nw + 127) / 128, 128, 0, st>>>(blk_idx, blk_cnt, topk, n_heads, n_qtiles, nb, plan, cnt,
+                                                     stride);
+    return cudaGetLastError();
+}
+
+cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, const int *s_idx, int n_slash,
+                        int n, int n_heads, int n_qtiles, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(b.bits_v, 0, sizeof(uint32_t) * (size_t)n_heads * b.words, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b.bits_s, 0, sizeof(uint32_t) * (size_t)n_heads * b.words, st);
+    if (e != cudaSuccess) return e;
+    vs_mark_kernel<<<n_heads, 256, 0, st>>>(v_idx, n_vertical, s_idx, n_slash, n, b.bits_v, b.bits_s, b.words);
+    vs_extract_kernel<<<n_heads, 32, 0, st>>>(b.bits_v, b.bits_s, b.words, b.vsorted, b.nvs, b.vcap, b.soff,
+                                              b.scap, b.groups, b.ngroups);
+    const int nw = n_heads * n_qtiles;
+    vs_workitem_kernel<<<(nw + 3) / 4, 128, 0, st>>>(b.vsorted, b.nvs, b.vcap, b.groups, b.ngroups, b.scap,
+                                                     b.bits_s, b.words, n, n_heads, n_qtiles, b.nsh, b.nvert,
+                                                     b.vlist);
+    return cudaGetLastError();
+}
+
+}  // namespace minf

@@ -1,0 +1,82 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace minf {
+
+struct AttnParams;
+
+// Device buffers of the Vertical-Slash tile plan (all inside the workspace).
+struct VsPlanBufs {
+    uint32_t *bits_v, *bits_s;  // [n_heads][words]
+    int words;
+    int *vsorted, *nvs;         // [n_heads][vcap], [n_heads]
+    int vcap;
+    int *soff;                  // [n_heads][scap]
+    int2 *groups;               // [n_heads][scap]
+    int *ngroups;               // [n_heads]
+    int scap;
+    int *nsh, *nvert;           // [n_work]
+    int *vlist;                 // [n_work][vcap]
+};
+
+// 3D TMA map over a bf16 [heads][n][128] tensor: box {64, 64, 1}, 128B swizzle.
+cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n);
+
+cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st);
+cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_heads, int n_qtiles, int nb,
+                        int *plan, int *cnt, int stride, cudaStream_t st);
+cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, const int *s_idx, int n_slash,
+                        int n, int n_heads, int n_qtiles, cudaStream_t st);
+
+// Vertical-Slash estimation.
+struct VsEstBufs {
+    float2 *part;   // [n_pairs][n_chunks][128] running (max, sum) per row, log2 domain
+    float *lse2;    // [n_pairs][128]
+    float *diag;    // [n_heads][n_ktiles][191] per key-tile diagonal partial sums
+    float *vert;    // [n_heads][n]
+    float *slash;   // [n_heads][n]
+    int n_chunks, chunk_tiles, n_ktiles;
+};
+
+struct VsEstArgs {
+    const void *q, *k;     // bf16
+    int hq, hkv, n, last_q, n_heads;
+    float scale_log2;
+    const int *head_ids;   // host, n_heads entries
+    int n_vertical, n_slash;
+    int *v_idx, *s_idx;
+    void *hdr;             // WsHeader*
+    unsigned long long wait_limit_ns;
+};
+
+cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t st);
+
+// Block-Sparse estimation.
+struct BsEstBufs {
+    float *qp;       // [n_heads][nb][128]
+    float *kp;       // [hkv][nb][128]
+    float *scores;   // [head_batch][nb][nb]
+    int head_batch;
+};
+
+struct BsEstArgs {
+    const void *q, *k;
+    int hq, hkv, n, n_heads, topk;
+    const int *head_ids;  // host
+    int *blk_idx, *blk_cnt;
+};
+
+cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStream_t st);
+
+// Self-test of the bounded wait.
+cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaStream_t st);
+
+// Top-k (largest first, ties to the lower index) of n_rows rows of `len`
+// non-negative floats each; writes min(k, len) indices ascending, -1 padded to k.
+cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, cudaStream_t st);
+
+}  // namespace minf

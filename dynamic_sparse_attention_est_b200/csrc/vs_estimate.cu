@@ -1,0 +1,329 @@
+// vs_estimate.cu -- Vertical-Slash index estimation on sm_100a.
+//
+// News article "单卡A100实现百万token推理，速度快10倍，这是微软官方的大模型推理加速",
+// section 方法介绍: the vertical and slash indices of a head are estimated from
+// the attention of its last queries against all keys.  Here, per q-head:
+//   pass 1  lse_i  = log-sum-exp over keys k <= i of scale * q_i . k_k, for the
+//           last 64 rows i (split over key chunks, then combined);
+//   pass 2  A_ik   = exp(scale * q_i . k_k - lse_i), summed along columns
+//           (vertical score of key k) and along diagonals (slash score of the
+//           offset o = i - k);
+//   top-k   the best keys and offsets (radix select, ties to the lower index),
+//           offset 0 forced.
+// Both passes run S = Q K^T on the tensor cores: one CTA holds the last 64 rows
+// of two q-heads of the same kv-head as one M=128 tile (TMEM lanes 0-63 and
+// 64-127) and streams 128-key tiles of K through TMA.  Pass 2 reduces the
+// softmax weights through a skewed shared-memory buffer, so that column and
+// diagonal sums come out deterministic and without atomics.
+#include <cfloat>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace minf {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr uint32_t kTileBytes = 32768;
+constexpr int kDiagW = 191;          // offsets one 128-key tile touches for 64 rows
+constexpr int kSkewRows = 95;        // offsets one 32-key chunk touches for 64 rows
+constexpr int kSkewStride = 65;      // padded row stride (floats) of the skew buffer
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kTileBytes;
+constexpr uint32_t kSmemSkew = kSmemK + kStages * kTileBytes;                 // 2*95*65 floats
+constexpr uint32_t kSmemDiag = kSmemSkew + 2 * kSkewRows * kSkewStride * 4;  // 2*191 floats
+constexpr uint32_t kSmemBar = (kSmemDiag + 2 * kDiagW * 4 + 255) & ~255u;
+constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;
+
+enum : int { B_Q = 0, B_KF = 1, B_KE = 4, B_SF = 7, B_SE = 9, B_COUNT = 11 };
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, false);
+
+struct EstParams {
+    CUtensorMap tmap_q, tmap_k;
+    int4 pairs[MINF_MAX_HEADS];  // (hp0, hp1, h0, h1); hp1 = -1 when the second half is empty
+    int n_pairs, n, group, last_q, n_ktiles, chunk_tiles, n_chunks;
+    float scale_log2;
+    float2 *part;
+    const float *lse2;
+    float *vert, *diag;
+    int *status;
+    unsigned long long wait_limit_ns;
+};
+
+template <int MODE>  // 0: per-row (max, sum) partials; 1: column and diagonal sums
+__global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_constant__ EstParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sQ = smem_u32(smem) + kSmemQ, sK = smem_u32(smem) + kSmemK;
+    float *skew = reinterpret_cast<float *>(smem + kSmemSkew);
+    float *tdiag = reinterpret_cast<float *>(smem + kSmemDiag);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + B_COUNT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT + 1);
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = blockIdx.x % P.n_pairs, chunk = blockIdx.x / P.n_pairs;
+    const int4 pr = P.pairs[pair];
+    const int g = pr.z / P.group;
+    const int kt0 = chunk * P.chunk_tiles;
+    const int T = max(0, min(P.chunk_tiles, P.n_ktiles - kt0));
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_Q), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(B_KF + s), 1);
+            mbar_init(bar(B_KE + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_SF + b), 1);
+            mbar_init(bar(B_SE + b), 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl wc{abort_flag, P.status, P.wait_limit_ns};
+
+    if (warp == 0) {
+        if (lane == 0 && T > 0) {
+            const int q0 = P.n - 64;
+            const int h1 = pr.y >= 0 ? pr.w : pr.z;
+            mbar_expect_tx(bar(B_Q), 4 * 8192);
+            tma_load_3d(sQ, &P.tmap_q, bar(B_Q), 0, q0, pr.z);
+            tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q), 64, q0, pr.z);
+            tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q), 0, q0, h1);
+            tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q), 64, q0, h1);
+            mbar_arrive(bar(B_Q));
+            for (int j = 0; j < T; ++j) {
+                const int s = j % kStages;
+                if (!wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc)) break;
+                const uint32_t st = sK + s * kTileBytes;
+                const int key0 = (kt0 + j) * 128;
+                mbar_expect_tx(bar(B_KF + s), kTileBytes);
+                tma_load_3d(st, &P.tmap_k, bar(B_KF + s), 0, key0, g);
+                tma_load_3d(st + 16384, &P.tmap_k, bar(B_KF + s), 64, key0, g);
+                tma_load_3d(st + 8192, &P.tmap_k, bar(B_KF + s), 0, key0 + 64, g);
+                tma_load_3d(st + 16384 + 8192, &P.tmap_k, bar(B_KF + s), 64, key0 + 64, g);
+                mbar_arrive(bar(B_KF + s));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && T > 0) {
+            bool ok = wait_bounded(bar(B_Q), 0, wc);
+            if (ok) tc_fence_after();
+            for (int j = 0; ok && j < T; ++j) {
+                const int s = j % kStages, b = j & 1;
+                if (!wait_bounded(bar(B_KF + s), (j / kStages) & 1, wc)) break;
+                if (!wait_bounded(bar(B_SE + b), ((j >> 1) & 1) ^ 1, wc)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tmem + b * 128, sdesc_sw128(sQ + off, 16, 1024),
+                            sdesc_sw128(sK + s * kTileBytes + off, 16, 1024), kIdescQK, kk != 0);
+                }
+                umma_commit(bar(B_KE + s));
+                umma_commit(bar(B_SF + b));
+            }
+        }
+    } else if (warp >= 4) {
+        const int r = threadIdx.x - 128;
+        const int rr = r & 63, hh = r >> 6;
+        const int i = P.n - 64 + rr;  // query position of this row
+        const bool head_ok = hh == 0 || pr.y >= 0;
+        const bool row_ok = head_ok && rr >= 64 - P.last_q;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const float sl2 = P.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
+        float lse2 = 0.f;
+        if constexpr (MODE == 1) lse2 = row_ok ? P.lse2[pair * 128 + r] : 0.f;
+        if (MODE == 1 && !(lse2 > -INFINITY)) lse2 = 0.f;
+        for (int j = 0; j < T; ++j) {
+            const int b = j & 1;
+            const int kt = kt0 + j;
+            const bool got = wait_bounded(bar(B_SF + b), (j >> 1) & 1, wc);
+            // one decision for all 128 threads: the reduction below uses named barriers
+            if (named_bar_or(1, 128, !got || *abort_flag)) break;
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + b * 128 + c * 32, sr[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+            tc_fence_before();
+            mbar_arrive(bar(B_SE + b));
+            const int cmax = row_ok ? i - kt * 128 : -1;  // columns c <= cmax are keys <= i
+            if constexpr (MODE == 0) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c * 32 + e <= cmax) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+                mx *= sl2;
+                const float m_new = fmaxf(m_run, mx);
+                if (m_new > -INFINITY) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (c * 32 + e <= cmax)
+                                acc += ex2_approx(fmaf(__uint_as_float(sr[c][e]), sl2, -m_new));
+                    l_run = l_run * ex2_approx(m_run - m_new) + acc;
+                    m_run = m_new;
+                }
+            } else {
+                // zero this tile's diagonal accumulator
+                for (int x = r; x < 2 * kDiagW; x += 128) tdiag[x] = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    named_bar_sync(1, 128);  // previous readers of the skew buffer are done
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float p = (cc * 32 + c <= cmax)
+                                            ? ex2_approx(fmaf(__uint_as_float(sr[cc][c]), sl2, -lse2))
+                                            : 0.f;
+                        skew[(hh * kSkewRows + (rr - c + 31)) * kSkewStride + rr] = p;
+                    }
+                    named_bar_sync(1, 128);
+                    for (int task = r; task < 64 + 2 * kSkewRows; task += 128) {
+                        if (task < 64) {  // column sum of one key over the 64 rows of one head
+                            const int h2 = task >> 5, c = task & 31;
+                            float s = 0.f;
+                            for (int r2 = 0; r2 < 64; ++r2) s += skew[(h2 * kSkewRows + (r2 - c + 31)) * kSkewStride + r2];
+                            const int key = kt * 128 + cc * 32 + c;
+                            const int hp2 = h2 == 0 ? pr.x : pr.y;
+                            if (hp2 >= 0 && key < P.n) P.vert[(size_t)hp2 * P.n + key] = s;
+                        } else {  // diagonal sum of one offset
+                            const int t2 = task - 64;
+                            const int h2 = t2 / kSkewRows, orel = t2 % kSkewRows;
+                            float s = 0.f;
+                            const int lo = max(0, orel - 31), hi = min(63, orel);
+                            for (int r2 = lo; r2 <= hi; ++r2) s += skew[(h2 * kSkewRows + orel) * kSkewStride + r2];
+                            tdiag[h2 * kDiagW + orel + 96 - 32 * cc] += s;
+                        }
+                    }
+                }
+                named_bar_sync(1, 128);
+                for (int x = r; x < 2 * kDiagW; x += 128) {
+                    const int h2 = x / kDiagW;
+                    const int hp2 = h2 == 0 ? pr.x : pr.y;
+                    if (hp2 >= 0) P.diag[((size_t)hp2 * P.n_ktiles + kt) * kDiagW + (x % kDiagW)] = tdiag[x];
+                }
+                named_bar_sync(1, 128);
+            }
+        }
+        if constexpr (MODE == 0) {
+            P.part[((size_t)pair * P.n_chunks + chunk) * 128 + r] = make_float2(m_run, l_run);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// lse2[pair][row] = log2 sum over chunks of the partial (max, sum) pairs.
+__global__ void lse_combine_kernel(const float2 *part, int n_pairs, int n_chunks, float *lse2) {
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= n_pairs * 128) return;
+    const int pair = x / 128, r = x % 128;
+    float m = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) m = fmaxf(m, part[((size_t)pair * n_chunks + c) * 128 + r].x);
+    float l = 0.f;
+    if (m > -INFINITY)
+        for (int c = 0; c < n_chunks; ++c) {
+            const float2 p = part[((size_t)pair * n_chunks + c) * 128 + r];
+            if (p.x > -INFINITY) l += p.y * exp2f(p.x - m);
+        }
+    lse2[x] = l > 0.f ? m + log2f(l) : -INFINITY;
+}
+
+// slash[hp][o] = sum of the (at most two) key tiles' diagonal partials that
+// cover offset o, in increasing tile order; offset 0 is forced to +inf.
+__global__ void slash_combine_kernel(const float *diag, int n, int n_ktiles, float *slash) {
+    const int hp = blockIdx.y;
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o >= n) return;
+    float s = 0.f;
+    const int hi = min(n_ktiles - 1, (n - 1 - o) >> 7);  // last tile whose keys can sit o before a row
+    for (int kt = max(0, hi - 2); kt <= hi; ++kt) {
+        const int rel = o - (n - kDiagW - kt * 128);
+        if (rel >= 0 && rel < kDiagW) s += diag[((size_t)hp * n_ktiles + kt) * kDiagW + rel];
+    }
+    slash[(size_t)hp * n + o] = o == 0 ? INFINITY : s;
+}
+
+}  // namespace
+
+cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t st) {
+    EstParams P;
+    memset(&P, 0, sizeof(P));
+    cudaError_t e = make_tmap_3d(&P.tmap_q, a.q, a.hq, a.n);
+    if (e == cudaSuccess) e = make_tmap_3d(&P.tmap_k, a.k, a.hkv, a.n);
+    if (e != cudaSuccess) return e;
+    const int group = a.hq / a.hkv;
+    // pair the listed heads that share a kv-head: M = 128 rows = 2 x 64 rows
+    int np = 0;
+    for (int g = 0; g < a.hkv; ++g) {
+        int pending = -1;
+        for (int hp = 0; hp < a.n_heads; ++hp) {
+            const int h = a.head_ids[hp];
+            if (h / group != g) continue;
+            if (pending < 0) {
+                pending = hp;
+            } else {
+                P.pairs[np++] = make_int4(pending, hp, a.head_ids[pending], h);
+                pending = -1;
+            }
+        }
+        if (pending >= 0) P.pairs[np++] = make_int4(pending, -1, a.head_ids[pending], a.head_ids[pending]);
+    }
+    P.n_pairs = np;
+    P.n = a.n;
+    P.group = group;
+    P.last_q = a.last_q;
+    P.n_ktiles = b.n_ktiles;
+    P.chunk_tiles = b.chunk_tiles;
+    P.n_chunks = b.n_chunks;
+    P.scale_log2 = a.scale_log2;
+    P.part = b.part;
+    P.lse2 = b.lse2;
+    P.vert = b.vert;
+    P.diag = b.diag;
+    P.status = a.hdr ? &reinterpret_cast<WsHeader *>(a.hdr)->status : nullptr;
+    P.wait_limit_ns = a.wait_limit_ns;
+    if (np == 0) return cudaSuccess;
+
+    e = cudaFuncSetAttribute(vs_est_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(vs_est_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = np * b.n_chunks;
+    vs_est_kernel<0><<<grid, kThreads, kSmemBytes, st>>>(P);
+    lse_combine_kernel<<<(np * 128 + 255) / 256, 256, 0, st>>>(b.part, np, b.n_chunks, b.lse2);
+    vs_est_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(P);
+    dim3 sg((a.n + 255) / 256, a.n_heads);
+    slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, st);
+    if (e != cudaSuccess) return e;
+    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, st);
+}
+
+}  // namespace minf

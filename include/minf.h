@@ -1,0 +1,220 @@
+/*
+ * minf.h -- C ABI of the B200 (sm_100a) dynamic sparse prefill attention library.
+ *
+ * The library implements the online half of MInference-style dynamic sparse
+ * attention for the long-context pre-filling stage: per-head sparse-index
+ * estimation (Vertical-Slash, Block-Sparse) and the causal sparse attention
+ * that consumes the indices (Vertical-Slash, Block-Sparse, A-shape), plus a
+ * dense causal attention kernel used as the comparison baseline.
+ *
+ * Sources (page title, section):
+ *   [NEWS] "单卡A100实现百万token推理，速度快10倍，这是微软官方的大模型推理加速"
+ *          (yntaolf.cn), section 方法介绍 -- the three patterns; Vertical-Slash
+ *          indices estimated from the attention of the last queries against all
+ *          keys; Block-Sparse indices from mean-pooled Q and K multiplied
+ *          (pooling commutes with the product); block-sparse FlashAttention.
+ *          Section 延迟和内核中的稀疏模式, Figure 4 -- inside the kernel the
+ *          verticals are 1x64 pieces and the slashes 64x64 blocks.
+ *   [TALK] "以 KV 缓存为中心的高效长文本方法" (AICon 2025 talk transcript,
+ *          dify360.com), second observation -- A-shape (initial tokens plus a
+ *          local window), vertical lines, slash lines, block clusters; the
+ *          offline/online split with per-head patterns.
+ *
+ * Conventions shared by every call:
+ *   - Tensors are CALLER-OWNED DEVICE buffers on one CUDA device; the library
+ *     allocates no device memory.  Scratch space is the caller's `ws` buffer of
+ *     at least minf_workspace_bytes(...) bytes (256-byte aligned).
+ *   - q is bf16 [hq][n][128], k and v are bf16 [hkv][n][128], row-major and
+ *     contiguous; d must be 128.  GQA: q-head h reads kv-head h / (hq / hkv).
+ *   - n must be a positive multiple of 64 (MINF_ERR_UNSUPPORTED otherwise).
+ *   - head_ids is an optional HOST array of n_heads q-head ids (distinct, each
+ *     in [0, hq)); NULL means every head, n_heads = hq.  Outputs are indexed by
+ *     position in that list: out [n_heads][n][128] bf16, lse [n_heads][n] fp32
+ *     (natural log of the softmax denominator; -inf for a row with no key).
+ *     At most MINF_MAX_HEADS heads per call.
+ *   - scale multiplies q.k before the softmax and must be > 0 (1/sqrt(128) is
+ *     the usual value).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t); the return value
+ *     reports argument checks and launch errors only.  A device-side failure
+ *     (a bounded wait that ran out) is recorded in the workspace status word and
+ *     read back by minf_status().
+ *   - Causal masking throughout: query i sees keys k <= i only.
+ *
+ * Return codes: MINF_OK, or a negative MINF_ERR_* value; arguments are checked
+ * on the host before anything is launched, so an error return launches nothing.
+ */
+#ifndef MINF_H
+#define MINF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t minf_bf16;                /* raw bf16 bits */
+typedef struct CUstream_st *minf_stream_t; /* the same type as cudaStream_t */
+
+#define MINF_OK 0
+#define MINF_ERR_INVALID (-1)     /* null pointer, hq % hkv != 0, budget < 1, bad head id, scale <= 0 */
+#define MINF_ERR_UNSUPPORTED (-2) /* d != 128, n % 64 != 0, block != 64, last_q > 64, no sm_100 device */
+#define MINF_ERR_CUDA (-3)        /* a CUDA runtime/driver call or launch failed */
+#define MINF_ERR_TIMEOUT (-4)     /* a device-side bounded wait gave up (see minf_status) */
+#define MINF_ERR_WORKSPACE (-5)   /* ws_bytes smaller than minf_workspace_bytes(...) */
+
+#define MINF_MAX_HEADS 256
+
+/* Operation codes for minf_workspace_bytes. */
+#define MINF_OP_VS_ESTIMATE 1
+#define MINF_OP_VS_ATTENTION 2
+#define MINF_OP_BLOCK_ESTIMATE 3
+#define MINF_OP_BLOCK_ATTENTION 4
+#define MINF_OP_ASHAPE_ATTENTION 5
+#define MINF_OP_DENSE_ATTENTION 6
+#define MINF_OP_MIXED_LAYER 7
+
+/* Per-head pattern codes for minf_mixed_layer. */
+#define MINF_PATTERN_DENSE 0
+#define MINF_PATTERN_VS 1
+#define MINF_PATTERN_BLOCK 2
+#define MINF_PATTERN_ASHAPE 3
+
+/*
+ * Bytes of workspace an operation needs.  p1/p2/p3 by op:
+ *   VS_ESTIMATE, VS_ATTENTION: p1 = n_vertical, p2 = n_slash
+ *   BLOCK_ESTIMATE, BLOCK_ATTENTION: p1 = topk
+ *   MIXED_LAYER: p1 = n_vertical, p2 = n_slash, p3 = topk (n_heads ignored: all hq heads)
+ *   others: unused.
+ * Returns 0 for arguments the op would reject.
+ */
+size_t minf_workspace_bytes(int op, int hq, int hkv, int n, int n_heads, int p1, int p2, int p3);
+
+/*
+ * Vertical-Slash index estimation ([NEWS] 方法介绍).  For each listed q-head,
+ * the softmax rows of the last `last_q` queries (causal, keys k <= i) are
+ * summed along columns (vertical score of key k) and along diagonals (slash
+ * score of offset o = i - k).  Offset 0 is forced into the slash set and takes
+ * one slot.  The best min(n_vertical, n) keys and min(n_slash, n) offsets are
+ * kept, ties to the lower index, and written ASCENDING:
+ *   v_idx int32 [n_heads][n_vertical], s_idx int32 [n_heads][n_slash],
+ *   each row padded with -1 past its min(budget, n) valid entries.
+ * 1 <= last_q <= 64.
+ */
+int minf_vs_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                     int last_q, int n_vertical, int n_slash, float scale,
+                     const int32_t *head_ids, int n_heads, int32_t *v_idx, int32_t *s_idx,
+                     void *ws, size_t ws_bytes, minf_stream_t stream);
+
+/*
+ * Vertical-Slash sparse attention.  Query i of head position p attends to
+ * key k iff k <= i and (k is in v_idx[p] or i - k is in s_idx[p]); each such
+ * key once.  Entries < 0 in the index rows are ignored; rows need not be
+ * sorted.  Slash lines are computed as contiguous key ranges per 128-query
+ * tile ([NEWS] Figure 4: slashes as dense blocks), verticals outside those
+ * ranges are gathered by index ([NEWS] Figure 4: verticals as 1x64 pieces).
+ */
+int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv,
+                      int n, int d, float scale, const int32_t *head_ids, int n_heads,
+                      const int32_t *v_idx, int n_vertical, const int32_t *s_idx, int n_slash,
+                      minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                      minf_stream_t stream);
+
+/*
+ * Block-Sparse index estimation ([NEWS] 方法介绍).  Q and K are mean-pooled
+ * over blocks of `block` (= 64) tokens in fp32; for query block i the pooled
+ * score of key block j <= i is Qp_i . Kp_j.  The diagonal block i is always
+ * kept; the best topk-1 blocks j < i join it (ties to the lower j).  Output,
+ * ASCENDING, -1 padded:
+ *   blk_idx int32 [n_heads][n/64][topk], blk_cnt int32 [n_heads][n/64].
+ */
+int minf_block_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                        int block, int topk, const int32_t *head_ids, int n_heads,
+                        int32_t *blk_idx, int32_t *blk_cnt, void *ws, size_t ws_bytes,
+                        minf_stream_t stream);
+
+/*
+ * Block-Sparse attention: query i of head position p attends to key k iff
+ * k <= i and k / 64 is among blk_idx[p][i / 64][0 .. blk_cnt[p][i / 64]).
+ * Each row of blk_idx must be ascending with distinct entries (as
+ * minf_block_estimate writes it); negative entries are ignored.
+ */
+int minf_block_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
+                         int hkv, int n, int d, float scale, const int32_t *head_ids,
+                         int n_heads, const int32_t *blk_idx, const int32_t *blk_cnt, int topk,
+                         minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                         minf_stream_t stream);
+
+/*
+ * A-shape attention ([TALK] second observation): query i attends to key k iff
+ * k <= i and (k < n_sink or i - k < window).  The window counts the query
+ * itself.  n_sink >= 0, window >= 1.
+ */
+int minf_ashape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
+                          int hkv, int n, int d, float scale, const int32_t *head_ids,
+                          int n_heads, int n_sink, int window, minf_bf16 *out, float *lse,
+                          void *ws, size_t ws_bytes, minf_stream_t stream);
+
+/* Dense causal attention (the comparison baseline): query i attends to k <= i. */
+int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
+                         int hkv, int n, int d, float scale, const int32_t *head_ids,
+                         int n_heads, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                         minf_stream_t stream);
+
+/*
+ * One attention layer with a per-head pattern ([TALK] offline/online split:
+ * each head has its own pattern; the online part estimates and attends).
+ * head_pattern is a HOST array of hq MINF_PATTERN_* codes.  VS heads run
+ * minf_vs_estimate + minf_vs_attention (last_q, n_vertical, n_slash), BLOCK
+ * heads minf_block_estimate + minf_block_attention (64, topk), ASHAPE heads
+ * minf_ashape_attention (n_sink, window), DENSE heads minf_dense_attention.
+ * out [hq][n][128] bf16, lse [hq][n] fp32 (nullable).  The indices are kept in
+ * the workspace; everything runs on `stream`.
+ */
+int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv,
+                     int n, int d, float scale, const int8_t *head_pattern, int last_q,
+                     int n_vertical, int n_slash, int topk, int n_sink, int window,
+                     minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                     minf_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the device-side status word of the
+ * workspace: MINF_OK, or MINF_ERR_TIMEOUT if a bounded wait in a kernel gave up
+ * (that kernel then left its outputs incomplete).  Reading it resets it to
+ * MINF_OK.  Returns MINF_ERR_CUDA if the synchronisation itself failed.
+ */
+int minf_status(void *ws, minf_stream_t stream);
+
+/*
+ * Synchronises `stream` and returns the work counters the last attention call
+ * on `ws` accumulated: tiles = 128x128 query-key tiles computed on the tensor
+ * cores, pairs = (query, key) pairs inside the mask (the useful work).
+ */
+int minf_stats(void *ws, minf_stream_t stream, uint64_t *tiles, uint64_t *pairs);
+
+/*
+ * Sets the limit, in nanoseconds, after which a device-side wait gives up and
+ * records MINF_ERR_TIMEOUT (default 2e9 ns; 0 restores the default).  Applies
+ * to launches made after the call, process-wide.
+ */
+void minf_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Failure-detection self-test: launches one kernel whose wait nothing will
+ * ever satisfy, so it must give up after `limit_ns` and record
+ * MINF_ERR_TIMEOUT in the workspace status word (read with minf_status).
+ * Needs MINF_STATUS_BYTES of workspace.
+ */
+int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_stream_t stream);
+
+#define MINF_STATUS_BYTES 256
+
+/* Library version string and the message of the last host-side error. */
+const char *minf_version(void);
+const char *minf_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MINF_H */

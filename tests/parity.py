@@ -1,0 +1,68 @@
+"""Comparison rules of the CUDA path against the fp64 oracle.
+
+* Attention outputs (oracle indices fed to both sides): max |gpu - oracle|
+  <= 2e-2 and mean |gpu - oracle| <= 2e-3 on bf16 inputs; the log-sum-exp
+  within 1e-2 absolute (fp32 accumulation, ex2.approx).
+* Index sets: with t the oracle's k-th best score, every item scoring above
+  t + band is in the GPU set, every item below t - band is not, and the set
+  holds exactly k items; band = 1e-3 |t| + 1e-6 (the relative 1e-3 tie band,
+  with an absolute floor for scores that sit near zero).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+LSE_ABS = 1e-2
+REL_BAND = 1e-3
+ABS_BAND = 1e-6
+
+
+def to_np(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().numpy().astype(np.float64)
+    return np.asarray(t, dtype=np.float64)
+
+
+def check_attention(gpu_out, gpu_lse, ref_out, ref_lse, what=""):
+    g = to_np(gpu_out)
+    r = np.asarray(ref_out, np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU output"
+    err = np.abs(g - r)
+    assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
+    if gpu_lse is not None and ref_lse is not None:
+        gl = to_np(gpu_lse)
+        rl = np.asarray(ref_lse, np.float64)
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(gl), fin), f"{what}: lse finiteness differs"
+        if fin.any():
+            le = np.abs(gl[fin] - rl[fin]).max()
+            assert le <= LSE_ABS, f"{what}: lse max abs err {le:.3e}"
+    return float(err.max()), float(err.mean())
+
+
+def check_topk_band(gpu_idx, scores, k, what=""):
+    """gpu_idx: 1-D indices (-1 padded); scores: oracle fp64 scores of every candidate."""
+    scores = np.asarray(scores, np.float64)
+    kk = min(k, len(scores))
+    got = [int(x) for x in np.asarray(gpu_idx).ravel() if x >= 0]
+    assert len(got) == kk, f"{what}: {len(got)} indices, expected {kk}"
+    assert len(set(got)) == kk, f"{what}: duplicate indices"
+    assert got == sorted(got), f"{what}: not ascending"
+    if kk == 0:
+        return 0
+    order = np.sort(scores)[::-1]
+    t = order[kk - 1]
+    band = REL_BAND * abs(t) + ABS_BAND if np.isfinite(t) else 0.0
+    gs = set(got)
+    must = np.nonzero(scores > t + band)[0]
+    never = np.nonzero(scores < t - band)[0]
+    miss = [int(i) for i in must if int(i) not in gs]
+    extra = [int(i) for i in never if int(i) in gs]
+    assert not miss, f"{what}: missing clear winners {miss[:10]}"
+    assert not extra, f"{what}: took clear losers {extra[:10]}"
+    return len(got) - len(set(must.tolist()) & gs)  # picks decided inside the band

@@ -1,0 +1,187 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Sizes here are small enough for the oracle to finish in seconds, yet span
+several 128-row tiles and ragged tails (n % 128 == 64).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_sparse_attention_est_b200 import minf, synth
+from parity import check_attention, check_topk_band, to_np
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+def inputs(n, hq, hkv, structure="vertical", seed=0, n_heavy=8):
+    w = synth.Workload("test", "vs", hq, hkv, n, structure, n_heavy=n_heavy)
+    x = synth.generate(w, seed=seed)
+    return x["q"], x["k"], x["v"]
+
+
+def cuda(*ts):
+    return [t.cuda() for t in ts]
+
+
+@pytest.mark.parametrize("n,hq,hkv", [(128, 1, 1), (320, 1, 1), (1024, 4, 2), (1088, 2, 2)])
+def test_dense(orc, n, hq, hkv):
+    q, k, v = inputs(n, hq, hkv, seed=n)
+    ref, rl = orc.dense_attention(q, k, v, SCALE)
+    out, lse = minf.minf_dense_attention(*cuda(q, k, v), scale=SCALE)
+    check_attention(out, lse, ref, rl, f"dense n={n}")
+
+
+def test_dense_head_subset(orc):
+    q, k, v = inputs(576, 4, 2, seed=3)
+    ids = [3, 0]
+    ref, rl = orc.dense_attention(q, k, v, SCALE, head_ids=ids)
+    out, lse = minf.minf_dense_attention(*cuda(q, k, v), scale=SCALE, head_ids=ids)
+    check_attention(out, lse, ref, rl, "dense subset")
+
+
+@pytest.mark.parametrize("sink,window", [(128, 256), (100, 300), (0, 1), (64, 5000), (7, 64)])
+def test_ashape(orc, sink, window):
+    n = 1344
+    q, k, v = inputs(n, 2, 1, structure="plain", seed=sink + window)
+    ref, rl = orc.ashape_attention(q, k, v, SCALE, sink, window)
+    out, lse = minf.minf_ashape_attention(*cuda(q, k, v), n_sink=sink, window=window, scale=SCALE)
+    check_attention(out, lse, ref, rl, f"A-shape {sink}/{window}")
+
+
+@pytest.mark.parametrize("topk", [1, 4, 16])
+def test_block_attention_oracle_indices(orc, topk):
+    n = 1216
+    q, k, v = inputs(n, 4, 2, structure="plain", seed=topk)
+    bi, bc = orc.block_estimate(q, k, 64, topk)
+    ref, rl = orc.block_attention(q, k, v, SCALE, 64, bi, bc)
+    out, lse = minf.minf_block_attention(*cuda(q, k, v), torch.from_numpy(bi).cuda(), torch.from_numpy(bc).cuda(),
+                                         scale=SCALE)
+    check_attention(out, lse, ref, rl, f"block topk={topk}")
+
+
+def test_block_estimate_band(orc):
+    n = 2048
+    w = synth.Workload("t", "block", 4, 2, n, "clustered")
+    x = synth.generate(w, seed=1)
+    q, k = x["q"], x["k"]
+    topk = 8
+    bi, bc, _, _, sc = orc.block_estimate(q, k, 64, topk, return_scores=True)
+    gi, gc = minf.minf_block_estimate(*cuda(q, k), topk=topk)
+    gi, gc = gi.cpu().numpy(), gc.cpu().numpy()
+    nb = n // 64
+    for hp in range(4):
+        for i in range(nb):
+            row = gi[hp, i, :gc[hp, i]]
+            assert gc[hp, i] == min(topk, i + 1)
+            assert row[-1] == i, "diagonal block forced"
+            check_topk_band(row[:-1], sc[hp, i, :i], topk - 1, f"block row {hp}/{i}")
+            assert np.all(gi[hp, i, gc[hp, i]:] == -1)
+
+
+def _rand_vs_indices(rng, n, nh, nv, ns):
+    vi = np.full((nh, nv), -1, np.int32)
+    si = np.full((nh, ns), -1, np.int32)
+    for hp in range(nh):
+        a = rng.choice(n, nv - 3, replace=False)
+        vi[hp, :nv - 3] = a[rng.permutation(len(a))]           # unsorted
+        vi[hp, nv - 3] = a[0]                                    # a duplicate
+        b = rng.choice(n, ns - 2, replace=False)
+        si[hp, :ns - 2] = b
+    return vi, si
+
+
+@pytest.mark.parametrize("n,hq,hkv,nv,ns", [(1024, 4, 2, 40, 60), (1344, 2, 1, 100, 30), (4096, 1, 1, 256, 512)])
+def test_vs_attention_oracle_indices(orc, n, hq, hkv, nv, ns):
+    q, k, v = inputs(n, hq, hkv, seed=nv)
+    vi, si = orc.vs_estimate(q, k, 64, nv, ns, SCALE)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out, lse, ref, rl, f"VS n={n}")
+
+
+def test_vs_attention_unsorted_duplicate_indices(orc):
+    n, hq, hkv = 1088, 2, 1
+    q, k, v = inputs(n, hq, hkv, seed=77)
+    vi, si = _rand_vs_indices(np.random.default_rng(5), n, hq, 50, 70)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out, lse, ref, rl, "VS random sets")
+
+
+@pytest.mark.parametrize("n,hq,hkv,last_q,nv,ns", [(4096, 1, 1, 64, 256, 512), (2048, 4, 2, 64, 100, 300),
+                                                   (1088, 3, 1, 17, 30, 40)])
+def test_vs_estimate_band(orc, n, hq, hkv, last_q, nv, ns):
+    q, k, _ = inputs(n, hq, hkv, seed=n + hq)
+    vi, si, vert, slash = orc.vs_estimate(q, k, last_q, nv, ns, SCALE, return_scores=True)
+    gv, gs = minf.minf_vs_estimate(*cuda(q, k), last_q=last_q, n_vertical=nv, n_slash=ns, scale=SCALE)
+    gv, gs = gv.cpu().numpy(), gs.cpu().numpy()
+    for hp in range(hq):
+        check_topk_band(gv[hp], vert[hp], nv, f"vertical h{hp}")
+        check_topk_band(gs[hp], slash[hp], ns, f"slash h{hp}")
+        assert 0 in set(gs[hp].tolist()), "offset 0 forced"
+
+
+def test_vs_end_to_end_4k(orc):
+    """4K single head, planted verticals: GPU estimate, then GPU attention on the GPU's indices vs the
+    oracle attention on the same indices."""
+    w = synth.WORKLOADS["vs-1h-4k"]
+    x = synth.generate(w, seed=0)
+    q, k, v = x["q"], x["k"], x["v"]
+    gv, gs = minf.minf_vs_estimate(*cuda(q, k), last_q=64, n_vertical=256, n_slash=512, scale=SCALE)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), gv, gs, scale=SCALE)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, gv.cpu().numpy(), gs.cpu().numpy())
+    check_attention(out, lse, ref, rl, "VS 4k end to end")
+
+
+def test_mixed_layer(orc):
+    n, hq, hkv = 1280, 8, 2
+    q, k, v = inputs(n, hq, hkv, seed=11)
+    pats = ["vs", "block", "ashape", "dense", "vs", "vs", "block", "ashape"]
+    nv, ns, topk, sink, window = 40, 80, 6, 64, 256
+    out, lse = minf.minf_mixed_layer(*cuda(q, k, v), pats, last_q=64, n_vertical=nv, n_slash=ns, topk=topk,
+                                     n_sink=sink, window=window, scale=SCALE)
+    for h, p in enumerate(pats):
+        ids = [h]
+        if p == "vs":
+            vi, si = orc.vs_estimate(q, k, 64, nv, ns, SCALE, head_ids=ids)
+            ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si, head_ids=ids)
+        elif p == "block":
+            bi, bc = orc.block_estimate(q, k, 64, topk, head_ids=ids)
+            ref, rl = orc.block_attention(q, k, v, SCALE, 64, bi, bc, head_ids=ids)
+        elif p == "ashape":
+            ref, rl = orc.ashape_attention(q, k, v, SCALE, sink, window, head_ids=ids)
+        else:
+            ref, rl = orc.dense_attention(q, k, v, SCALE, head_ids=ids)
+        check_attention(out[h:h + 1], lse[h:h + 1], ref, rl, f"mixed head {h} ({p})")
+
+
+def test_stats_count_dense_tiles():
+    n, hq, hkv = 1088, 2, 1
+    q, k, v = cuda(*inputs(n, hq, hkv, seed=2))
+    ws = minf.workspace(256, q.device)
+    minf.minf_dense_attention(q, k, v, scale=SCALE, ws=ws)
+    tiles, pairs = minf.minf_stats(ws)
+    nt = (n + 127) // 128
+    halves = sum(min(2 * t + 2, n // 64) for t in range(nt))
+    assert tiles == hq * sum((min(2 * t + 2, n // 64) + 1) // 2 for t in range(nt))
+    assert pairs == hq * n * (n + 1) // 2
+    assert halves > 0
+    assert minf.minf_status(ws) == minf.MINF_OK
+
+
+def test_bounded_wait_reports_timeout():
+    ws = minf.workspace(256, torch.device("cuda"))
+    minf.minf_check_wait_timeout(ws, 2_000_000)  # 2 ms
+    assert minf.minf_status(ws) == minf.MINF_ERR_TIMEOUT
+    assert minf.minf_status(ws) == minf.MINF_OK  # reading resets it
+    # the context is still usable
+    q, k, v = cuda(*inputs(128, 1, 1, seed=0))
+    out, _ = minf.minf_dense_attention(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
