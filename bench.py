@@ -1,0 +1,423 @@
+"""Benchmark: dynamic sparse prefill attention (estimate + attention) per layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl minf|reference]
+
+A step is one pass of the whole path over one layer of synthetic input:
+  vs-gqa-32k       minf_vs_estimate + minf_vs_attention (32 q-heads / 8 kv-heads, 32K tokens)
+  block-gqa-128k   minf_block_estimate + minf_block_attention (128K tokens)
+  ashape-gqa-128k  minf_ashape_attention (128K tokens)
+  mixed-gqa-1m     minf_mixed_layer, per-head patterns drawn from the seed (1M tokens)
+The default is vs-gqa-32k.  Inputs stay resident in HBM and are larger than L2,
+so no flush is needed between steps.  The line also carries the roofline of the
+attention kernel (computed-tile FLOPs / its CUDA-event time), the same metric
+end to end from pinned host buffers, the dense causal kernel on the same
+inputs, and the fp64 CPU oracle timed on a bounded sample.
+
+With --gpus N (under torchrun), every rank runs its own layer (weak scaling,
+no collective on the data path); value = max-over-ranks time / layers run.
+``--impl reference`` times the fp64 oracle (the reference arm) on the host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill attention ms/layer"
+_T0 = time.time()
+
+
+def log(msg: str) -> None:
+    """Progress on stderr (the JSON line alone goes to stdout)."""
+    print(f"[bench {time.time() - _T0:7.1f}s] {msg}", file=sys.stderr, flush=True)
+UNIT = "ms/layer"
+TILE_FLOPS = 4 * 128 * 128 * 128  # QK^T and PV of one 128x128 tile, d = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="vs-gqa-32k")
+    ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-kernel comparison")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work to sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload
+def make_step(w, x, torch, minf, synth, seed):
+    """Returns (step(ws) -> out, attention-only call for timing, label of the attention call)."""
+    q, k, v = x["q"], x["k"], x["v"]
+    hq, hkv, n = w.hq, w.hkv, w.n
+    dev = q.device
+    scale = 1.0 / math.sqrt(128)
+    if w.pattern == "vs":
+        ws_est = minf.workspace(minf.workspace_bytes(minf.OP_VS_ESTIMATE, hq, hkv, n, hq), dev)
+        ws = minf.workspace(minf.workspace_bytes(minf.OP_VS_ATTENTION, hq, hkv, n, hq, w.n_vertical, w.n_slash),
+                            dev)
+        out = torch.empty_like(q)
+        state = {}
+
+        def estimate():
+            state["idx"] = minf.minf_vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, scale, ws=ws_est)
+
+        def attend():
+            vi, si = state["idx"]
+            minf.minf_vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
+
+        return estimate, attend, ws, out, 6, 4
+    if w.pattern == "block":
+        ws_est = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ESTIMATE, hq, hkv, n, hq, w.topk), dev)
+        ws = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ATTENTION, hq, hkv, n, hq, w.topk), dev)
+        out = torch.empty_like(q)
+        state = {}
+
+        def estimate():
+            state["idx"] = minf.minf_block_estimate(q, k, w.topk, ws=ws_est)
+
+        def attend():
+            bi, bc = state["idx"]
+            minf.minf_block_attention(q, k, v, bi, bc, scale, out=out, want_lse=False, ws=ws)
+
+        nbatch = math.ceil(hq / max(1, min(hq, (1 << 30) // ((n // 64) ** 2 * 4))))
+        return estimate, attend, ws, out, 2 + 2 * nbatch, 2
+    if w.pattern == "ashape":
+        ws = minf.workspace(256, dev)
+        out = torch.empty_like(q)
+
+        def attend():
+            minf.minf_ashape_attention(q, k, v, w.n_sink, w.window, scale, out=out, want_lse=False, ws=ws)
+
+        return (lambda: None), attend, ws, out, 0, 1
+    if w.pattern == "mixed":
+        pats = synth.mixed_head_patterns(w, seed)
+        ws = minf.workspace(minf.workspace_bytes(minf.OP_MIXED_LAYER, hq, hkv, n, hq, w.n_vertical, w.n_slash,
+                                                 w.topk), dev)
+        out = torch.empty_like(q)
+
+        def attend():
+            minf.minf_mixed_layer(q, k, v, pats, w.last_q, w.n_vertical, w.n_slash, w.topk, w.n_sink, w.window,
+                                  scale, out=out, want_lse=False, ws=ws)
+
+        return (lambda: None), attend, ws, out, 0, 16
+    raise ValueError(w.pattern)
+
+
+def cpu_sample(w, x, orc, budget_s, seed):
+    """Times the fp64 oracle on a bounded sample of the workload and scales it to one layer."""
+    import numpy as np
+    import torch
+
+    scale = 1.0 / math.sqrt(128)
+    hq, hkv, n = w.hq, w.hkv, w.n
+    g = hq // hkv
+    # one q-head (and its kv-head) as float32 host arrays
+    q1 = x["q"][0:1].float().cpu().numpy()
+    k1 = x["k"][0:1].float().cpu().numpy()
+    v1 = x["v"][0:1].float().cpu().numpy()
+    est_s = 0.0
+    detail = []
+    t0 = time.perf_counter()
+    if w.pattern in ("vs", "mixed"):
+        vi, si = orc.vs_estimate(q1, k1, w.last_q, w.n_vertical, w.n_slash, scale)
+        est_s = time.perf_counter() - t0
+        detail.append(f"VS estimate of 1 head ({est_s:.2f} s) x {hq}")
+    elif w.pattern == "block":
+        if n // 64 <= 4096:
+            bi, bc = orc.block_estimate(q1, k1, 64, w.topk)
+            est_s = time.perf_counter() - t0
+            detail.append(f"block estimate of 1 head ({est_s:.2f} s) x {hq}")
+    # attention rows: spread over the sequence, grown until the budget is used
+    rows_per_s = None
+    nrows = 64
+    spent = 0.0
+    while True:
+        rows = np.linspace(0, n - 1, nrows).astype(np.int32)
+        t1 = time.perf_counter()
+        if w.pattern in ("vs", "mixed"):
+            orc.vs_attention(q1, k1, v1, scale, vi, si, rows=rows)
+        elif w.pattern == "block":
+            if n // 64 > 4096:
+                bi = np.tile(np.arange(w.topk, dtype=np.int32), (1, n // 64, 1))
+                bc = np.full((1, n // 64), w.topk, np.int32)
+            orc.block_attention(q1, k1, v1, scale, 64, bi, bc, rows=rows)
+        else:
+            orc.ashape_attention(q1, k1, v1, scale, w.n_sink, w.window, rows=rows)
+        dt = time.perf_counter() - t1
+        spent += dt
+        rows_per_s = nrows / dt
+        if spent > budget_s * 0.5 or nrows >= n:
+            break
+        nrows = min(n, int(nrows * max(2.0, (budget_s * 0.5) / max(dt, 1e-3))))
+    attn_layer_s = hq * n / rows_per_s
+    layer_s = est_s * hq + attn_layer_s
+    detail.append(f"attention of {nrows} rows spread over the sequence of 1 head, scaled to {hq} x {n} rows")
+    return {"value": layer_s * 1000.0, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+            "sample": "; ".join(detail)}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from dynamic_sparse_attention_est_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle
+        import torch
+
+        orc = oracle.get()
+        # the sample attends with q-head 0 only: draw that head and its kv-head
+        x = synth.generate(w, seed=args.seed, device="cpu", hq=1, hkv=1)
+        per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+        vals = []
+        for i in range(args.warmup + args.steps):
+            r = cpu_sample(w, x, orc, per, args.seed)
+            if i >= args.warmup:
+                vals.append(r["value"])
+        val = statistics.median(vals)
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "hq": w.hq, "hkv": w.hkv, "n": w.n},
+                "cpu_baseline": {"value": val, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                                 "sample": r["sample"]},
+                "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    from dynamic_sparse_attention_est_b200 import minf
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    seed = args.seed + rank
+    log(f"generating {w.name} on {dev}")
+    x = synth.generate(w, seed=seed, device=dev)
+    torch.cuda.synchronize()
+    log("inputs ready")
+    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        estimate()
+        attend()
+
+    for i in range(max(3, args.warmup)):
+        estimate()
+        torch.cuda.synchronize()
+        log(f"warm-up {i}: estimate done")
+        attend()
+        torch.cuda.synchronize()
+        log(f"warm-up {i}: attention done")
+    tiles, pairs = minf.minf_stats(ws)
+    if minf.minf_status(ws) != minf.MINF_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- timed region: K steps, events around the whole and around each attention call
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        estimate()
+        ev[i][0].record(stream)
+        attend()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    elapsed = t_start.elapsed_time(t_end)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        elapsed = float(t.item())
+    ms_per_layer = elapsed / (args.steps * world)
+    ms_per_step = elapsed / args.steps
+
+    log(f"timed region done: {ms_per_layer:.3f} ms/layer")
+    # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        hq_, hk_, hv_ = (x["q"].cpu().pin_memory(), x["k"].cpu().pin_memory(), x["v"].cpu().pin_memory())
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        qd, kd, vd = x["q"], x["k"], x["v"]
+        e2e_steps = max(2, min(args.steps, 5))
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            qd.copy_(hq_, non_blocking=True)
+            kd.copy_(hk_, non_blocking=True)
+            vd.copy_(hv_, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        h2d = hq_.numel() * 2 + hk_.numel() * 2 + hv_.numel() * 2
+        e2e = {"value": a.elapsed_time(b) / e2e_steps, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": host_out.numel() * 2}
+
+    log("end-to-end timing done")
+    # ---- dense kernel on the same inputs (context for the sparse speedup)
+    dense = None
+    if not args.no_dense and w.n <= 131072:
+        wsd = minf.workspace(256, dev)
+        outd = torch.empty_like(x["q"])
+        minf.minf_dense_attention(x["q"], x["k"], x["v"], out=outd, want_lse=False, ws=wsd)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        a.record(stream)
+        for _ in range(reps):
+            minf.minf_dense_attention(x["q"], x["k"], x["v"], out=outd, want_lse=False, ws=wsd)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dtiles, _ = minf.minf_stats(wsd)
+        dms = a.elapsed_time(b) / reps
+        dense = {"ms_per_layer": dms, "tflops_computed": dtiles * TILE_FLOPS / (dms * 1e-3) / 1e12,
+                 "sparse_speedup": dms / ms_per_layer * world}
+
+    peaks, src = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    achieved = tiles * TILE_FLOPS / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "attn_kernel (timed with its plan kernels, CUDA events around the attention call)",
+                "peak_source": f"{src} bf16_tflops_sustained"}
+
+    log("dense comparison done")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
+
+        xs = {"q": x["q"][:1].cpu(), "k": x["k"][:1].cpu(), "v": x["v"][:1].cpu()}
+        cpu = cpu_sample(w, xs, oracle.get(), args.cpu_budget, seed)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(ms_per_layer, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; RoPE'd N(0,1) with planted structure)",
+            "config": {"workload": w.name, "pattern": w.pattern, "hq": w.hq, "hkv": w.hkv, "n": w.n,
+                       "last_q": w.last_q, "n_vertical": w.n_vertical, "n_slash": w.n_slash, "topk": w.topk,
+                       "n_sink": w.n_sink, "window": w.window,
+                       "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"one layer per rank x{world}"},
+            "roofline": roofline,
+            "attention_ms": round(attn_ms, 4),
+            "estimate_ms": round(ms_per_step - attn_ms, 4),
+            "computed_tiles": tiles, "mask_pairs": pairs,
+            "useful_tflops": round(4 * 128 * pairs / (attn_ms * 1e-3) / 1e12, 1),
+            "dense": dense,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": (n_est_k + n_att_k) * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -628,14 +628,16 @@ int minf_status(void *ws, minf_stream_t stream) {
     if (!ws) return fail(MINF_ERR_INVALID, "null workspace");
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    int status = 0;
-    e = cudaMemcpy(&status, ws, sizeof(int), cudaMemcpyDeviceToHost);
+    int st[2] = {0, 0};
+    e = cudaMemcpy(st, ws, sizeof(st), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy status");
-    if (status != 0) {
-        e = cudaMemset(ws, 0, sizeof(int));
+    if (st[0] != 0) {
+        fail(st[0], "device wait gave up at site 0x%08x (role %d, barrier %d, tile %d)", st[1],
+             (st[1] >> 24) & 0x3f, (st[1] >> 16) & 0xff, st[1] & 0xffff);
+        e = cudaMemset(ws, 0, sizeof(st));
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemset status");
     }
-    return status;
+    return st[0];
 }
 
 int minf_stats(void *ws, minf_stream_t stream, uint64_t *tiles, uint64_t *pairs) {

@@ -310,7 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             HalfDesc hd[2];
             hd[0] = gen.next(P);
             hd[1] = gen.next(P);
-            if (!wait_bounded(bar(empty0 + s), ph ^ 1, wc)) break;
+            // one decision per warp: every lane takes the same path through load_tile
+            const bool got = wait_bounded(bar(empty0 + s), ph ^ 1, wc, wait_site(is_k ? 1 : 2, empty0 + s, j));
+            if (__any_sync(0xffffffffu, !got)) break;
             load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
             issued = j + 1;
         }
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const uint32_t tP[2] = {tmem + 384, tmem + 448};
             auto issue_s = [&](int j) -> bool {
                 const int s = j & 1;
-                if (!wait_bounded(bar(B_K_FULL + s), (j >> 1) & 1, wc)) return false;
+                if (!wait_bounded(bar(B_K_FULL + s), (j >> 1) & 1, wc, wait_site(3, B_K_FULL + s, j))) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 umma_commit(bar(B_S_FULL + s));
                 return true;
             };
-            bool ok = wait_bounded(bar(B_Q_FULL), 0, wc);
+            bool ok = wait_bounded(bar(B_Q_FULL), 0, wc, wait_site(3, B_Q_FULL, 0));
             if (ok) {
                 tc_fence_after();
                 ok = issue_s(0);
@@ -351,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             for (int j = 0; ok && j < T; ++j) {
                 const int b = j & 1;
                 const uint32_t ph = (j >> 1) & 1;
-                if (!wait_bounded(bar(B_P_FULL + b), ph, wc)) break;
-                if (!wait_bounded(bar(B_V_FULL + b), ph, wc)) break;
+                if (!wait_bounded(bar(B_P_FULL + b), ph, wc, wait_site(3, B_P_FULL + b, j))) break;
+                if (!wait_bounded(bar(B_V_FULL + b), ph, wc, wait_site(3, B_V_FULL + b, j))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -390,7 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, bits_s, bits_v);
             const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, bits_s, bits_v);
             if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
-            if (!wait_bounded(bar(B_S_FULL + b), ph, wc)) { ok = false; break; }
+            const bool got = wait_bounded(bar(B_S_FULL + b), ph, wc, wait_site(4, B_S_FULL + b, j));
+            if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // tcgen05.ld below is warp-wide
             tc_fence_after();
             uint32_t sr[4][32];
 #pragma unroll
@@ -412,22 +415,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             mx *= sl2;
             const float m_new = fmaxf(m_run, mx);
-            if (m_new > m_run + 8.0f) {
-                const float alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
-                if (j > 0 && m_run != -INFINITY) {
-                    // O holds tiles < j: wait for P(j-1) V(j-1), then rescale it in TMEM
-                    if (!wait_bounded(bar(B_O_DONE), (j - 1) & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
+            const bool want = m_new > m_run + 8.0f;  // includes m_run = -inf with a finite m_new
+            const float alpha = want ? ex2_approx(m_run - m_new) : 1.f;  // 0 when m_run = -inf
+            // O (tiles < j) is rescaled in TMEM by the whole warp at once: tcgen05.ld/st are
+            // warp-collective, so lanes that keep their max take alpha = 1
+            if (j > 0 && __any_sync(0xffffffffu, want && m_run != -INFINITY)) {
+                const bool done = wait_bounded(bar(B_O_DONE), (j - 1) & 1, wc, wait_site(4, B_O_DONE, j));
+                if (__any_sync(0xffffffffu, !done)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-                        tmem_ld_wait(o);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait(o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tO + c * 32, o);
-                    }
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + c * 32, o);
                 }
+            }
+            if (want) {
                 l_run *= alpha;
                 m_run = m_new;
             }
@@ -463,7 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             mbar_arrive(bar(B_P_FULL + b));
         }
         // epilogue
-        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc, wait_site(4, B_ALL_DONE, T));
+        ok = __all_sync(0xffffffffu, ok);  // the epilogue's TMEM loads are warp-wide
         if (ok) {
             tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;

@@ -18,7 +18,7 @@ constexpr int kBlock = 64;     // Block-Sparse block size / Vertical-Slash row g
 // Workspace header: status word + counters, first 256 bytes of every workspace.
 struct WsHeader {
     int status;
-    int pad;
+    int site;  // where the first bounded wait gave up: role << 24 | barrier << 16 | tile
     unsigned long long tiles;
     unsigned long long pairs;
 };

@@ -58,11 +58,12 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
 // waiting too, and returns false.
 struct WaitCtl {
     volatile int *abort_flag;  // shared memory
-    int *status;               // global status word
+    int *status;               // global status word; status[1] records the site
     uint64_t limit_ns;
 };
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl &w) {
+// `site` identifies the wait (role << 24 | barrier << 16 | tile) for diagnosis.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl &w, int site = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -70,11 +71,18 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
         if (*w.abort_flag) return false;
         if (globaltimer_ns() - t0 > w.limit_ns) {
             *w.abort_flag = 1;
-            if (w.status) atomicExch(w.status, -4);
+            if (w.status) {
+                atomicExch(w.status, -4);
+                atomicCAS(w.status + 1, 0, site | 0x40000000);
+            }
             __threadfence();
             return false;
         }
     }
+}
+
+__host__ __device__ constexpr int wait_site(int role, int barrier, int tile) {
+    return (role << 24) | (barrier << 16) | (tile & 0xFFFF);
 }
 
 // --------------------------------------------------------------------- TMA

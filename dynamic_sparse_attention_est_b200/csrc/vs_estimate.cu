@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
             mbar_arrive(bar(B_Q));
             for (int j = 0; j < T; ++j) {
                 const int s = j % kStages;
-                if (!wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc)) break;
+                if (!wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc, wait_site(5, B_KE + s, j))) break;
                 const uint32_t st = sK + s * kTileBytes;
                 const int key0 = (kt0 + j) * 128;
                 mbar_expect_tx(bar(B_KF + s), kTileBytes);
@@ -122,12 +122,12 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
         }
     } else if (warp == 1) {
         if (lane == 0 && T > 0) {
-            bool ok = wait_bounded(bar(B_Q), 0, wc);
+            bool ok = wait_bounded(bar(B_Q), 0, wc, wait_site(6, B_Q, 0));
             if (ok) tc_fence_after();
             for (int j = 0; ok && j < T; ++j) {
                 const int s = j % kStages, b = j & 1;
-                if (!wait_bounded(bar(B_KF + s), (j / kStages) & 1, wc)) break;
-                if (!wait_bounded(bar(B_SE + b), ((j >> 1) & 1) ^ 1, wc)) break;
+                if (!wait_bounded(bar(B_KF + s), (j / kStages) & 1, wc, wait_site(6, B_KF + s, j))) break;
+                if (!wait_bounded(bar(B_SE + b), ((j >> 1) & 1) ^ 1, wc, wait_site(6, B_SE + b, j))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
             const int kt = kt0 + j;
-            const bool got = wait_bounded(bar(B_SF + b), (j >> 1) & 1, wc);
+            const bool got = wait_bounded(bar(B_SF + b), (j >> 1) & 1, wc, wait_site(7, B_SF + b, j));
             // one decision for all 128 threads: the reduction below uses named barriers
             if (named_bar_or(1, 128, !got || *abort_flag)) break;
             tc_fence_after();
