@@ -667,3 +667,74 @@ const char *minf_version(void) { return "minf-b200 0.1.0 (sm_100a)"; }
 const char *minf_last_error(void) { return g_last_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Vertical-Slash estimate without a caller workspace.
+//
+// Some callers cannot allocate device memory at the point where they estimate
+// indices -- for example code running inside a caller's own memory-managed
+// runtime or a capture region where cudaMalloc is not allowed, or an embedding
+// that has no allocator at all.  For them this entry point takes its scratch
+// from one file-scope device array of kNoAllocScratchBytes, which every GPU
+// that loads the library holds until the process exits.  Requests whose
+// scratch would exceed it are rejected with MINF_ERR_WORKSPACE.
+//
+// The array's device address is looked up once per device, by the first call
+// made on that device (with that device current); make that first call before
+// any stream capture.  Every call shares the array: calls whose work overlaps
+// on the GPU (different streams, or different host threads, with no ordering
+// between them) race on it.  The status block at its start is cleared by each
+// call; device-side timeouts are therefore not reported by this variant.
+namespace minf {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[64] = {nullptr};
+
+int noalloc_scratch(int dev, void **out) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+    if (dev < 0 || dev >= 64) return fail(MINF_ERR_UNSUPPORTED, "device %d out of range", dev);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MINF_OK;
+}
+
+}  // namespace
+}  // namespace minf
+
+extern "C" int minf_vs_estimate_noalloc(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                                        int last_q, int n_vertical, int n_slash, float scale,
+                                        const int32_t *head_ids, int n_heads, int32_t *v_idx, int32_t *s_idx,
+                                        minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v_idx || !s_idx) return fail(MINF_ERR_INVALID, "null v_idx or s_idx");
+    if (n_vertical < 1 || n_slash < 1) return fail(MINF_ERR_INVALID, "budgets must be >= 1");
+    if (last_q < 1) return fail(MINF_ERR_INVALID, "last_q must be >= 1");
+    if (last_q > 64) return fail(MINF_ERR_UNSUPPORTED, "last_q %d above 64", last_q);
+    const size_t need = bytes_vs_est(hkv, n, c.n_heads);
+    if (need > kNoAllocScratchBytes)
+        return fail(MINF_ERR_WORKSPACE, "needs %zu bytes of scratch; the built-in area holds %zu", need,
+                    kNoAllocScratchBytes);
+    if ((rc = select_device(q))) return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    void *ws = nullptr;
+    if ((rc = noalloc_scratch(dev, &ws))) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    e = cudaMemsetAsync(ws, 0, MINF_STATUS_BYTES, st);  // status block starts at zero
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+    return do_vs_estimate(c, q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws,
+                          static_cast<char *>(ws) + MINF_STATUS_BYTES, st);
+}

@@ -48,6 +48,7 @@ _SIGS = {
     "minf_ashape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "minf_dense_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_mixed_layer": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "minf_vs_estimate_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P]),
     "minf_status": (_I, [_P, _P]),
     "minf_stats": (_I, [_P, _P, ctypes.POINTER(_U64), ctypes.POINTER(_U64)]),
     "minf_set_wait_limit_ns": (None, [_U64]),
@@ -149,6 +150,23 @@ def minf_vs_estimate(q, k, last_q: int = 64, n_vertical: int = 1000, n_slash: in
     _check(lib().minf_vs_estimate(_ptr(q), _ptr(k), hq, hkv, n, d, last_q, n_vertical, n_slash, _scale(scale),
                                   ids, nh, _ptr(v_idx), _ptr(s_idx), _ptr(ws), ws.numel(), _stream(q.device)),
            "minf_vs_estimate")
+    return v_idx, s_idx
+
+
+def minf_vs_estimate_noalloc(q, k, last_q: int = 64, n_vertical: int = 1000, n_slash: int = 6096,
+                             scale: Optional[float] = None, head_ids=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """minf_vs_estimate with the library's built-in scratch instead of a workspace.
+
+    For callers that cannot allocate device memory for scratch; only the two
+    index outputs are allocated here (by torch, on behalf of this binding).
+    """
+    hq, hkv, n, d = _qkv(q, k)
+    ids, nh = _heads(hq, head_ids)
+    v_idx = torch.empty(nh, n_vertical, dtype=torch.int32, device=q.device)
+    s_idx = torch.empty(nh, n_slash, dtype=torch.int32, device=q.device)
+    _check(lib().minf_vs_estimate_noalloc(_ptr(q), _ptr(k), hq, hkv, n, d, last_q, n_vertical, n_slash,
+                                          _scale(scale), ids, nh, _ptr(v_idx), _ptr(s_idx), _stream(q.device)),
+           "minf_vs_estimate_noalloc")
     return v_idx, s_idx
 
 

@@ -209,6 +209,25 @@ int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_s
 
 #define MINF_STATUS_BYTES 256
 
+/*
+ * minf_vs_estimate without a workspace argument (no counterpart in the
+ * method's sources: it exists for callers that cannot allocate device memory,
+ * such as code inside a runtime that owns all device memory, or code that
+ * must not call cudaMalloc at that point).  Same arguments and results as
+ * minf_vs_estimate minus ws/ws_bytes; the scratch is a 32 MiB array inside
+ * the library that every GPU loading the library keeps until the process
+ * exits.  Calls needing more scratch than that (as sized by
+ * minf_workspace_bytes(MINF_OP_VS_ESTIMATE, ...)) return MINF_ERR_WORKSPACE.
+ * The first call on a device looks up the array's address on that device:
+ * make it before any stream capture.  All calls share the array, so calls
+ * that may overlap on the GPU race; order them on one stream.  Device-side
+ * timeouts are not reported by this variant.
+ */
+int minf_vs_estimate_noalloc(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                             int last_q, int n_vertical, int n_slash, float scale,
+                             const int32_t *head_ids, int n_heads, int32_t *v_idx, int32_t *s_idx,
+                             minf_stream_t stream);
+
 /* Library version string and the message of the last host-side error. */
 const char *minf_version(void);
 const char *minf_last_error(void);
