@@ -10,16 +10,21 @@
 // verticals as 1x64 pieces).  The pattern's exact mask is applied per element
 // inside each tile, so the result is the token-exact masked softmax.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer for Q and K (+ cp.async gathers of vertical keys)
-//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warp 2      TMA producer for V (+ gathers)
-//   warp 3      idle
-//   warps 4..7  softmax warpgroup: thread r owns query row r (TMEM lane r)
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
-// S = Q K^T (SS MMA), P = exp(S - m) as bf16 written back to TMEM, O += P V with
-// P read from TMEM (TS MMA).  Online softmax in fp32 with lazy rescaling: the
-// running max only moves when a row's max grows by more than 2^8.
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0       TMA producer for Q and K (+ cp.async gathers of vertical keys)
+//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma
+//   warp 2       TMA producer for V (+ gathers)
+//   warp 3       idle
+//   warps 4..7   softmax warpgroup 0: even key tiles
+//   warps 8..11  softmax warpgroup 1: odd key tiles
+// Thread r of a softmax warpgroup owns query row r (TMEM lane r).  TMEM
+// columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); each warpgroup
+// keeps its own running max, sum and O over its half of the key tiles, and
+// the two halves are merged in the epilogue.  S = Q K^T (SS MMA); P = exp(S-m)
+// as bf16 overwrites the first 64 columns of its S buffer and feeds O += P V
+// straight from TMEM (TS MMA).  The running max only moves when a row's max
+// grows by more than 2^8.  A fixed share of the exponentials runs on the FMA
+// pipe (polynomial) to offload the MUFU unit.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -28,17 +33,28 @@ namespace minf {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kStages = 3;                 // K ring and V ring depth
 constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kTileBytes;
-constexpr uint32_t kSmemV = kSmemK + 2 * kTileBytes;
-constexpr uint32_t kSmemBar = kSmemV + 2 * kTileBytes;
+constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
+constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
 constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
+// Register split after setmaxnreg: the launch gives 384 threads x 168 registers;
+// the load/MMA warpgroup drops to 56, the two softmax warpgroups rise to 224
+// (128 x 56 + 256 x 224 = 384 x 168).
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsLoad = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(128 * kRegsLoad + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+// Every kEmuEvery-th column pair takes its exponential from the FMA-pipe
+// polynomial instead of MUFU ex2 (0 disables it).
+constexpr int kEmuEvery = 4;
 
 enum : int {
-    B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 3, B_V_FULL = 5, B_V_EMPTY = 7,
-    B_S_FULL = 9, B_P_FULL = 11, B_O_DONE = 13, B_ALL_DONE = 14, B_COUNT = 15
+    B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 4, B_V_FULL = 7, B_V_EMPTY = 10,
+    B_S_FULL = 13, B_P_FULL = 15, B_ALL_DONE = 17, B_COUNT = 18
 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, false);
@@ -233,6 +249,28 @@ __device__ __forceinline__ void load_tile(uint32_t stage, uint32_t bar, const Ha
     if (lane == 0) mbar_arrive(bar);
 }
 
+// Exponential of a pair of arguments on the FMA pipe (Cody-Waite reduction for
+// base 2: x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f from a degree-3
+// minimax polynomial derived by csrc/exp2_poly.py, max relative error 7.5e-5;
+// 2^n assembled in the exponent bits).  Arguments at or below -127 give 0.
+__device__ __forceinline__ void exp2_poly_pair(float &a, float &b) {
+    const uint64_t magic = f32x2_splat(12582912.0f);  // 1.5 * 2^23: rounds to an integer in the low bits
+    uint64_t x = f32x2_pack(fmaxf(a, -127.f), fmaxf(b, -127.f));
+    const uint64_t t = f32x2_add(x, magic);
+    const uint64_t rn = f32x2_sub(t, magic);
+    const uint64_t f = f32x2_sub(x, rn);
+    uint64_t p = f32x2_fma(f, f32x2_splat(5.517166853e-02f), f32x2_splat(2.426111251e-01f));
+    p = f32x2_fma(p, f, f32x2_splat(6.932609677e-01f));
+    p = f32x2_fma(p, f, f32x2_splat(9.999280572e-01f));
+    float t0, t1;
+    f32x2_unpack(t, t0, t1);
+    // bits(2^n) = (n + 127) << 23 = bits(t) * 2^23 + 0x3F800000 (mod 2^32): n = -127 gives +0
+    const uint32_t s0 = __float_as_uint(t0) * (1u << 23) + 0x3F800000u;
+    const uint32_t s1 = __float_as_uint(t1) * (1u << 23) + 0x3F800000u;
+    p = f32x2_mul(p, f32x2_pack(__uint_as_float(s0), __uint_as_float(s1)));
+    f32x2_unpack(p, a, b);
+}
+
 template <int PAT>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
     extern __shared__ uint8_t smem_raw[];
@@ -253,15 +291,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q_FULL), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(B_K_FULL + s), 1);
             mbar_init(bar(B_K_EMPTY + s), 1);
             mbar_init(bar(B_V_FULL + s), 1);
             mbar_init(bar(B_V_EMPTY + s), 1);
-            mbar_init(bar(B_S_FULL + s), 1);
-            mbar_init(bar(B_P_FULL + s), 128);
         }
-        mbar_init(bar(B_O_DONE), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_S_FULL + b), 1);
+            mbar_init(bar(B_P_FULL + b), 128);
+        }
         mbar_init(bar(B_ALL_DONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -287,61 +326,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const int *vlist = nullptr;
     if constexpr (PAT == PAT_VS) vlist = P.vs_vert + (size_t)w_item * P.vs_vstride;
 
-    if (warp == 0 || warp == 2) {
-        // ------------------------------------------------------------ producers
-        const bool is_k = warp == 0;
-        const CUtensorMap *map = is_k ? &P.tmap_k : &P.tmap_v;
-        const __nv_bfloat16 *raw = is_k ? P.k : P.v;
-        const uint32_t stage0 = is_k ? sK : sV;
-        const int full0 = is_k ? B_K_FULL : B_V_FULL, empty0 = is_k ? B_K_EMPTY : B_V_EMPTY;
-        if (is_k && lane == 0 && T > 0) {
-            const int r0 = t * kTileM;
-            mbar_expect_tx(bar(B_Q_FULL), 4 * 8192);
-            tma_load_3d(sQ, &P.tmap_q, bar(B_Q_FULL), 0, r0, h);
-            tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q_FULL), 64, r0, h);
-            tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q_FULL), 0, r0 + 64, h);
-            tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q_FULL), 64, r0 + 64, h);
-            mbar_arrive(bar(B_Q_FULL));
-        }
-        int issued = 0;
-        for (int j = 0; j < T; ++j) {
-            const int s = j & 1;
-            const uint32_t ph = (j >> 1) & 1;
-            HalfDesc hd[2];
-            hd[0] = gen.next(P);
-            hd[1] = gen.next(P);
-            // one decision per warp: every lane takes the same path through load_tile
-            const bool got = wait_bounded(bar(empty0 + s), ph ^ 1, wc, wait_site(is_k ? 1 : 2, empty0 + s, j));
-            if (__any_sync(0xffffffffu, !got)) break;
-            load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
-            issued = j + 1;
-        }
-        if (*abort_flag && lane == 0) {
-            // drain: let the loads already issued land before the CTA exits
-            WaitCtl drain{abort_flag, nullptr, 50000000ull};
-            volatile int no_abort = 0;
-            drain.abort_flag = &no_abort;
-            for (int j = max(0, issued - 2); j < issued; ++j)
-                wait_bounded(bar(full0 + (j & 1)), (j >> 1) & 1, drain);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && T > 0) {
-            const uint32_t tS[2] = {tmem + 0, tmem + 128};
-            const uint32_t tO = tmem + 256;
-            const uint32_t tP[2] = {tmem + 384, tmem + 448};
+    if (warp < 4) {
+        // ---------------------------------------------------------- load / MMA warpgroup
+        setmaxnreg_dec<kRegsLoad>();
+        if (warp == 0 || warp == 2) {
+            const bool is_k = warp == 0;
+            const CUtensorMap *map = is_k ? &P.tmap_k : &P.tmap_v;
+            const __nv_bfloat16 *raw = is_k ? P.k : P.v;
+            const uint32_t stage0 = is_k ? sK : sV;
+            const int full0 = is_k ? B_K_FULL : B_V_FULL, empty0 = is_k ? B_K_EMPTY : B_V_EMPTY;
+            if (is_k && lane == 0 && T > 0) {
+                const int r0 = t * kTileM;
+                mbar_expect_tx(bar(B_Q_FULL), 4 * 8192);
+                tma_load_3d(sQ, &P.tmap_q, bar(B_Q_FULL), 0, r0, h);
+                tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q_FULL), 64, r0, h);
+                tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q_FULL), 0, r0 + 64, h);
+                tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q_FULL), 64, r0 + 64, h);
+                mbar_arrive(bar(B_Q_FULL));
+            }
+            int issued = 0;
+            for (int j = 0; j < T; ++j) {
+                const int s = j % kStages;
+                const uint32_t ph = (j / kStages) & 1;
+                HalfDesc hd[2];
+                hd[0] = gen.next(P);
+                hd[1] = gen.next(P);
+                // one decision per warp: every lane takes the same path through load_tile
+                const bool got = wait_bounded(bar(empty0 + s), ph ^ 1, wc, wait_site(is_k ? 1 : 2, empty0 + s, j));
+                if (__any_sync(0xffffffffu, !got)) break;
+                load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
+                issued = j + 1;
+            }
+            if (*abort_flag && lane == 0) {
+                // drain: let the loads already issued land before the CTA exits
+                volatile int no_abort = 0;
+                const WaitCtl drain{&no_abort, nullptr, 50000000ull};
+                for (int j = max(0, issued - kStages); j < issued; ++j)
+                    wait_bounded(bar(full0 + j % kStages), (j / kStages) & 1, drain);
+            }
+        } else if (warp == 1 && lane == 0 && T > 0) {
+            // tcgen05 issue: S(j) = Q K(j)^T into S[j % 2]; O[j % 2] += P(j) V(j) with P(j)
+            // read from the first 64 columns of S[j % 2]; S(j + 2) is issued after P(j) V(j)
+            // and the tensor pipe runs them in order, so P(j) is consumed before it is overwritten.
             auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!wait_bounded(bar(B_K_FULL + s), (j >> 1) & 1, wc, wait_site(3, B_K_FULL + s, j))) return false;
+                const int s = j % kStages;
+                if (!wait_bounded(bar(B_K_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j)))
+                    return false;
                 tc_fence_after();
+                const uint32_t dS = tmem + (j & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tS[s], sdesc_sw128(sQ + off, 16, 1024),
-                            sdesc_sw128(sK + s * kTileBytes + off, 16, 1024), kIdescQK, kk != 0);
+                    umma_ss(dS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + s * kTileBytes + off, 16, 1024),
+                            kIdescQK, kk != 0);
                 }
                 umma_commit(bar(B_K_EMPTY + s));
-                umma_commit(bar(B_S_FULL + s));
+                umma_commit(bar(B_S_FULL + (j & 1)));
                 return true;
             };
             bool ok = wait_bounded(bar(B_Q_FULL), 0, wc, wait_site(3, B_Q_FULL, 0));
@@ -351,31 +391,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (ok && T > 1) ok = issue_s(1);
             }
             for (int j = 0; ok && j < T; ++j) {
-                const int b = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!wait_bounded(bar(B_P_FULL + b), ph, wc, wait_site(3, B_P_FULL + b, j))) break;
-                if (!wait_bounded(bar(B_V_FULL + b), ph, wc, wait_site(3, B_V_FULL + b, j))) break;
+                const int b = j & 1, s = j % kStages;
+                if (!wait_bounded(bar(B_P_FULL + b), (j >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j))) break;
+                if (!wait_bounded(bar(B_V_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j))) break;
                 tc_fence_after();
+                const uint32_t dO = tmem + 256 + b * 128, aP = tmem + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tO, tP[b] + kk * 8, sdesc_sw128(sV + b * kTileBytes + kk * 2048, 16384, 1024),
-                            kIdescPV, (j | kk) != 0);
-                umma_commit(bar(B_V_EMPTY + b));
-                umma_commit(bar(B_O_DONE));
+                    umma_ts(dO, aP + kk * 8, sdesc_sw128(sV + s * kTileBytes + kk * 2048, 16384, 1024), kIdescPV,
+                            (j >= 2 || kk > 0) ? 1u : 0u);
+                umma_commit(bar(B_V_EMPTY + s));
                 if (j + 2 < T && !issue_s(j + 2)) break;
             }
-            // always close: the epilogue (or the abort path) waits for this
-            umma_commit(bar(B_ALL_DONE));
+            umma_commit(bar(B_ALL_DONE));  // always close: the epilogue (or the abort path) waits on it
             if (P.hdr) atomicAdd(&P.hdr->tiles, (unsigned long long)T);
         }
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ softmax
-        const int r = threadIdx.x - 128;
+    } else {
+        // ---------------------------------------------------------- softmax warpgroups
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int wg = (warp - 4) >> 2;          // 0: even tiles, 1: odd tiles
+        const int r = (threadIdx.x - 128) & 127; // query row = TMEM lane
         const int q = t * kTileM + r;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS[2] = {tmem + lane_off + 0, tmem + lane_off + 128};
-        const uint32_t tO = tmem + lane_off + 256;
-        const uint32_t tP[2] = {tmem + lane_off + 384, tmem + lane_off + 448};
+        const uint32_t tS = tmem + lane_off + wg * 128;
+        const uint32_t tO = tmem + lane_off + 256 + wg * 128;
         const float sl2 = P.scale_log2;
         const uint32_t *bits_s = nullptr, *bits_v = nullptr;
         if constexpr (PAT == PAT_VS) {
@@ -385,44 +424,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         float m_run = -INFINITY, l_run = 0.f;
         unsigned long long pairs = 0;
         bool ok = true;
-        for (int j = 0; j < T && ok; ++j) {
-            const int b = j & 1;
-            const uint32_t ph = (j >> 1) & 1;
-            HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
+        if (wg == 1) {  // tile 0 belongs to the other warpgroup
+            gen.next(P);
+            gen.next(P);
+        }
+        for (int j = wg; j < T; j += 2) {
+            const HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
+            gen.next(P);  // the other warpgroup's tile j + 1
+            gen.next(P);
             const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, bits_s, bits_v);
             const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, bits_s, bits_v);
+            const bool full = (hd0.flags & hd1.flags & HF_FULL) != 0;  // uniform over the CTA
             if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
-            const bool got = wait_bounded(bar(B_S_FULL + b), ph, wc, wait_site(4, B_S_FULL + b, j));
+            const bool got = wait_bounded(bar(B_S_FULL + wg), (j >> 1) & 1, wc, wait_site(4 + wg, B_S_FULL + wg, j));
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // tcgen05.ld below is warp-wide
             tc_fence_after();
             uint32_t sr[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS[b] + c * 32, sr[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-            float mx = -INFINITY;
+            if (!full) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint64_t mk = c < 2 ? mk0 : mk1;
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t mw = (uint32_t)((c < 2 ? mk0 : mk1) >> ((c & 1) * 32));
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int bit = (c & 1) * 32 + e;
-                    float x = __uint_as_float(sr[c][e]);
-                    x = ((mk >> bit) & 1ull) ? x : -INFINITY;
-                    sr[c][e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                    for (int e = 0; e < 32; ++e)
+                        if (!((mw >> e) & 1u)) sr[c][e] = 0xff800000u;  // -inf
                 }
             }
+            // row max over the 128 columns (three-input max)
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    mx = fmax3(mx, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
             mx *= sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool want = m_new > m_run + 8.0f;  // includes m_run = -inf with a finite m_new
             const float alpha = want ? ex2_approx(m_run - m_new) : 1.f;  // 0 when m_run = -inf
-            // O (tiles < j) is rescaled in TMEM by the whole warp at once: tcgen05.ld/st are
-            // warp-collective, so lanes that keep their max take alpha = 1
-            if (j > 0 && __any_sync(0xffffffffu, want && m_run != -INFINITY)) {
-                const bool done = wait_bounded(bar(B_O_DONE), (j - 1) & 1, wc, wait_site(4, B_O_DONE, j));
-                if (__any_sync(0xffffffffu, !done)) { ok = false; break; }
-                tc_fence_after();
+            // O[wg] holds this warpgroup's tiles < j, all complete (S(j) was issued after their P.V):
+            // rescale it in TMEM with the whole warp (lanes that keep their max use alpha = 1)
+            if (j >= 2 && __any_sync(0xffffffffu, want && m_run != -INFINITY)) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -438,69 +482,91 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 m_run = m_new;
             }
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            float lsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_use));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_use));
-                    lsum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
-                // reuse the first 16 registers of sr[c] as the packed row chunk
-#pragma unroll
-                for (int e = 0; e < 16; ++e) sr[c][e] = pk[e];
-            }
-            l_run += lsum;
+            const uint64_t sl2x2 = f32x2_splat(sl2), negm = f32x2_splat(-m_use);
+            uint64_t acc0 = 0, acc1 = 0;  // two running (sum, sum) pairs
             uint32_t pp[2][32];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                pp[0][e] = sr[0][e];
-                pp[0][16 + e] = sr[1][e];
-                pp[1][e] = sr[2][e];
-                pp[1][16 + e] = sr[3][e];
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                                                 sl2x2, negm);
+                    float p0, p1;
+                    f32x2_unpack(x, p0, p1);
+                    if (kEmuEvery > 0 && (e % kEmuEvery) == kEmuEvery - 1) {
+                        exp2_poly_pair(p0, p1);
+                    } else {
+                        p0 = ex2_approx(p0);
+                        p1 = ex2_approx(p1);
+                    }
+                    if (e & 1) acc1 = f32x2_add(acc1, f32x2_pack(p0, p1));
+                    else acc0 = f32x2_add(acc0, f32x2_pack(p0, p1));
+                    pp[c >> 1][(c & 1) * 16 + e] = pack_bf16x2(p0, p1);
+                }
             }
-            tmem_st32(tP[b], pp[0]);
-            tmem_st32(tP[b] + 32, pp[1]);
+            float a0, a1, b0, b1;
+            f32x2_unpack(acc0, a0, a1);
+            f32x2_unpack(acc1, b0, b1);
+            l_run += (a0 + a1) + (b0 + b1);
+            tmem_st32(tS, pp[0]);       // P(j) over the first 64 columns of S[wg]
+            tmem_st32(tS + 32, pp[1]);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar(B_P_FULL + b));
+            mbar_arrive(bar(B_P_FULL + wg));
         }
-        // epilogue
+        // ------------------------------------------------------------ epilogue
         ok = __all_sync(0xffffffffu, ok);
-        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc, wait_site(4, B_ALL_DONE, T));
-        ok = __all_sync(0xffffffffu, ok);  // the epilogue's TMEM loads are warp-wide
+        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc, wait_site(4 + wg, B_ALL_DONE, T));
+        ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-wide
+        // exchange (max, sum) of the two halves of the key stream through shared memory
+        // (the K stages are idle once every MMA has completed)
+        float2 *ex = reinterpret_cast<float2 *>(smem + kSmemK);
+        ex[wg * 128 + r] = make_float2(m_run, l_run);
+        named_bar_sync(1, 256);
         if (ok) {
             tc_fence_after();
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            const float2 s0 = ex[r], s1 = ex[128 + r];
+            const float m = fmaxf(s0.x, s1.x);
+            const float a0 = s0.x == -INFINITY ? 0.f : ex2_approx(s0.x - m);
+            const float a1 = (T < 2 || s1.x == -INFINITY) ? 0.f : ex2_approx(s1.x - m);
+            const float l = s0.y * a0 + s1.y * a1;
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float w0 = a0 * inv_l, w1 = a1 * inv_l;
             const size_t orow = (size_t)P.out_slot[hp] * P.n + min(q, P.n - 1);
-            uint4 *dst = reinterpret_cast<uint4 *>(P.out + orow * kD);
+            uint4 *dst = reinterpret_cast<uint4 *>(P.out + orow * kD + wg * 64);
+            const uint32_t tO0 = tmem + lane_off + 256 + wg * 64, tO1 = tmem + lane_off + 384 + wg * 64;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                if (T > 0) {  // uniform over the CTA: every lane of the warp loads
-                    tmem_ld32(tO + c * 32, o);
-                    tmem_ld_wait(o);
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o0[32], o1[32];
+                if (T > 0) {  // uniform over the CTA
+                    tmem_ld32(tO0 + c * 32, o0);
+                    tmem_ld_wait(o0);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                    for (int e = 0; e < 32; ++e) o0[e] = 0u;
+                }
+                if (T > 1) {
+                    tmem_ld32(tO1 + c * 32, o1);
+                    tmem_ld_wait(o1);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o1[e] = 0u;
                 }
                 if (q < P.n) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
-                                            __uint_as_float(o[2 * e + 1]) * inv_l);
+                    for (int e = 0; e < 16; ++e) {
+                        const float v0 = __uint_as_float(o0[2 * e]) * w0 + __uint_as_float(o1[2 * e]) * w1;
+                        const float v1 = __uint_as_float(o0[2 * e + 1]) * w0 + __uint_as_float(o1[2 * e + 1]) * w1;
+                        pk[e] = pack_bf16x2(v0, v1);
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
-            if (q < P.n && P.lse)
-                P.lse[orow] =
-                    l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+            if (wg == 0 && q < P.n && P.lse)
+                P.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
         if (P.hdr) {
 #pragma unroll
@@ -694,6 +760,12 @@ cudaError_t launch_attn(const AttnParams &P, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<PAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
+    // setmaxnreg.inc waits for registers the launch reserved: refuse to launch a
+    // build whose register count at entry would make the split wait forever
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_kernel<PAT>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
     const int grid = P.n_heads * P.n_qtiles;
     if (grid == 0) return cudaSuccess;
     attn_kernel<PAT><<<grid, kThreads, kSmemBytes, st>>>(P);
