@@ -277,7 +277,9 @@ def main():
         from datetime import timedelta
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    seed = args.seed + rank
+    from dynamic_sparse_attention_est_b200 import shard
+
+    seed = shard.rank_seed(args.seed, rank)
     log(f"generating {w.name} on {dev}")
     x = synth.generate(w, seed=seed, device=dev)
     torch.cuda.synchronize()
@@ -322,10 +324,8 @@ def main():
     elapsed = t_start.elapsed_time(t_end)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = shard.max_over_ranks(elapsed, device=dev)
         dist.barrier()
-        elapsed = float(t.item())
     ms_per_layer = elapsed / (args.steps * world)
     ms_per_step = elapsed / args.steps
 
@@ -336,7 +336,7 @@ def main():
         hq_, hk_, hv_ = (x["q"].cpu().pin_memory(), x["k"].cpu().pin_memory(), x["v"].cpu().pin_memory())
         host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         qd, kd, vd = x["q"], x["k"], x["v"]
-        e2e_steps = max(2, min(args.steps, 5))
+        e2e_steps = max(2, min(args.steps, 5 if w.n <= 131072 else 2))
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -356,23 +356,29 @@ def main():
     log("end-to-end timing done")
     # ---- dense kernel on the same inputs (context for the sparse speedup)
     dense = None
-    if not args.no_dense and w.n <= 131072:
+    if not args.no_dense:
+        # at 1M tokens a dense layer takes seconds: time a few heads and scale by the head count
+        heads = None if w.n <= 131072 else list(range(min(4, w.hq)))
+        nh = w.hq if heads is None else len(heads)
         wsd = minf.workspace(256, dev)
-        outd = torch.empty_like(x["q"])
-        minf.minf_dense_attention(x["q"], x["k"], x["v"], out=outd, want_lse=False, ws=wsd)
+        outd = torch.empty((nh,) + tuple(x["q"].shape[1:]), dtype=x["q"].dtype, device=dev)
+        minf.minf_dense_attention(x["q"], x["k"], x["v"], head_ids=heads, out=outd, want_lse=False, ws=wsd)
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        reps = 3
+        reps = 3 if heads is None else 1
         a.record(stream)
         for _ in range(reps):
-            minf.minf_dense_attention(x["q"], x["k"], x["v"], out=outd, want_lse=False, ws=wsd)
+            minf.minf_dense_attention(x["q"], x["k"], x["v"], head_ids=heads, out=outd, want_lse=False, ws=wsd)
         b.record(stream)
         torch.cuda.synchronize()
         dtiles, _ = minf.minf_stats(wsd)
-        dms = a.elapsed_time(b) / reps
-        dense = {"ms_per_layer": dms, "tflops_computed": dtiles * TILE_FLOPS / (dms * 1e-3) / 1e12,
-                 "sparse_speedup": dms / ms_per_layer * world}
+        dms_timed = a.elapsed_time(b) / reps
+        dms = dms_timed * w.hq / nh
+        dense = {"ms_per_layer": dms, "tflops_computed": dtiles * TILE_FLOPS / (dms_timed * 1e-3) / 1e12,
+                 "sparse_speedup": dms / ms_per_layer * world, "heads_timed": nh,
+                 "scaled_from_heads": heads is not None}
+        del outd
 
     peaks, src = measured_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))

@@ -662,6 +662,14 @@ int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_s
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "wait check launch");
 }
 
+int minf_selftest_exp2(const float *x, float *y_poly, float *y_hw, int n, minf_stream_t stream) {
+    if (!x || !y_poly || !y_hw || n < 0) return fail(MINF_ERR_INVALID, "bad self-test arguments");
+    int rc = select_device(x);
+    if (rc) return rc;
+    cudaError_t e = run_exp2_selftest(x, y_poly, y_hw, n, (cudaStream_t)stream);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "exp2 self-test launch");
+}
+
 const char *minf_version(void) { return "minf-b200 0.1.0 (sm_100a)"; }
 
 const char *minf_last_error(void) { return g_last_error.c_str(); }

@@ -772,7 +772,27 @@ cudaError_t launch_attn(const AttnParams &P, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// Applies the attention kernel's two exponential paths to x: the FMA-pipe
+// polynomial and the MUFU ex2 (self-test of the polynomial against the hardware).
+__global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_hw, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+    y_hw[i] = ex2_approx(a);
+    if (i + 1 < n) y_hw[i + 1] = ex2_approx(b);
+    exp2_poly_pair(a, b);
+    y_poly[i] = a;
+    if (i + 1 < n) y_poly[i + 1] = b;
+}
+
 }  // namespace
+
+cudaError_t run_exp2_selftest(const float *x, float *y_poly, float *y_hw, int n, cudaStream_t st) {
+    const int pairs = (n + 1) / 2;
+    if (pairs == 0) return cudaSuccess;
+    exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y_poly, y_hw, n);
+    return cudaGetLastError();
+}
 
 cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st) {
     switch (pattern) {

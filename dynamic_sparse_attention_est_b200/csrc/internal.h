@@ -72,6 +72,9 @@ struct BsEstArgs {
 
 cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStream_t st);
 
+// Self-test of the attention kernel's exponentials (polynomial and MUFU).
+cudaError_t run_exp2_selftest(const float *x, float *y_poly, float *y_hw, int n, cudaStream_t st);
+
 // Self-test of the bounded wait.
 cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaStream_t st);
 

@@ -53,6 +53,7 @@ _SIGS = {
     "minf_stats": (_I, [_P, _P, ctypes.POINTER(_U64), ctypes.POINTER(_U64)]),
     "minf_set_wait_limit_ns": (None, [_U64]),
     "minf_check_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
+    "minf_selftest_exp2": (_I, [_P, _P, _P, _I, _P]),
     "minf_version": (ctypes.c_char_p, []),
     "minf_last_error": (ctypes.c_char_p, []),
 }
@@ -280,6 +281,15 @@ def minf_set_wait_limit_ns(ns: int) -> None:
 def minf_check_wait_timeout(ws: torch.Tensor, limit_ns: int) -> None:
     _check(lib().minf_check_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(ws.device)),
            "minf_check_wait_timeout")
+
+
+def minf_selftest_exp2(x: torch.Tensor):
+    """(polynomial 2^x, hardware 2^x) as the attention kernels compute them."""
+    x = x.to(torch.float32).contiguous()
+    y_poly, y_hw = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().minf_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_hw), x.numel(), _stream(x.device)),
+           "minf_selftest_exp2")
+    return y_poly, y_hw
 
 
 def minf_version() -> str:

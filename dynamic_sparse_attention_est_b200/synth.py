@@ -68,6 +68,9 @@ WORKLOADS: Dict[str, Workload] = {
                                 block=64, topk=100),
     "ashape-gqa-128k": Workload("ashape-gqa-128k", "ashape", 32, 8, 131072, "plain",
                                  n_sink=128, window=4096),
+    # one Vertical-Slash head at 1M tokens with the layer's budgets: a profiling-size case
+    "vs-1h-1m": Workload("vs-1h-1m", "vs", 1, 1, 1048576, "vertical", heavy_frac=0.005,
+                          last_q=64, n_vertical=1000, n_slash=6096),
     "mixed-gqa-1m": Workload("mixed-gqa-1m", "mixed", 32, 8, 1048576, "vertical",
                               heavy_frac=0.005, last_q=64, n_vertical=1000, n_slash=6096,
                               block=64, topk=100, n_sink=128, window=4096,

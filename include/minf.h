@@ -210,6 +210,15 @@ int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_s
 #define MINF_STATUS_BYTES 256
 
 /*
+ * Self-test of the exponentials inside the attention kernels (no counterpart
+ * in the method's sources): for n fp32 inputs x (device), writes 2^x from the
+ * FMA-pipe polynomial the softmax uses for a share of its columns (Cody-Waite
+ * reduction to [-1/2, 1/2] plus a degree-3 minimax polynomial; 0 for
+ * x <= -127) to y_poly, and from the hardware ex2.approx to y_hw.
+ */
+int minf_selftest_exp2(const float *x, float *y_poly, float *y_hw, int n, minf_stream_t stream);
+
+/*
  * minf_vs_estimate without a workspace argument (no counterpart in the
  * method's sources: it exists for callers that cannot allocate device memory,
  * such as code inside a runtime that owns all device memory, or code that

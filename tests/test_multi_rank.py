@@ -1,0 +1,78 @@
+"""The multi-rank path on CPU: two gloo ranks share the heads of one layer.
+
+Each rank attends its own shard of GQA groups (computed here with the fp64
+oracle standing in for the per-rank kernels), the shards are gathered, and the
+result must equal the single-process layer; the timing reduction returns the
+maximum over ranks.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from dynamic_sparse_attention_est_b200 import shard, synth
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, result_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+
+    w = synth.WORKLOADS["mixed-gqa-1m"]
+    pats = synth.mixed_head_patterns(w, seed=3, hq=8)
+    x = synth.generate(synth.Workload("mr", "vs", 8, 4, 256, "vertical", n_heavy=4), seed=5)
+    parts = shard.partition_heads(pats, 4, world)
+    mine = parts[rank]
+    orc = oracle.get()
+    out, _ = orc.dense_attention(x["q"], x["k"], x["v"], 0.088, head_ids=mine)
+    full = torch.zeros(8, 256, 128, dtype=torch.float64)
+    full[mine] = torch.from_numpy(out)
+    dist.all_reduce(full)  # shards are disjoint: the sum assembles the layer
+    t = shard.max_over_ranks(1.0 + rank)
+    if rank == 0:
+        ref, _ = orc.dense_attention(x["q"], x["k"], x["v"], 0.088)
+        np.save(result_path, np.array([np.abs(full.numpy() - ref).max(), t,
+                                       len(set(parts[0]) & set(parts[1])), sum(len(p) for p in parts)]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_assemble_the_layer(tmp_path):
+    res = str(tmp_path / "res.npy")
+    mp.start_processes(_worker, args=(2, _free_port(), res), nprocs=2, join=True, start_method="spawn")
+    err, tmax, overlap, total = np.load(res)
+    assert err == 0.0
+    assert tmax == 2.0
+    assert overlap == 0 and total == 8
+
+
+def test_partition_is_balanced_and_keeps_groups_whole():
+    w = synth.WORKLOADS["mixed-gqa-1m"]
+    pats = synth.mixed_head_patterns(w, seed=0)
+    for world in (1, 2, 4, 8):
+        parts = shard.partition_heads(pats, 8, world)
+        flat = sorted(h for p in parts for h in p)
+        assert flat == list(range(32))
+        for p in parts:
+            assert all(((h // 4) * 4 + i) in p for h in p for i in range(4))  # whole groups
+        loads = shard.shard_summary(parts, pats)
+        if world <= 8:
+            heaviest_group = max(sum(shard.PATTERN_COST[pats[g * 4 + i]] for i in range(4)) for g in range(8))
+            assert max(loads.values()) - min(loads.values()) <= heaviest_group + 1e-9
+
+
+def test_rank_seeds_differ():
+    assert len({shard.rank_seed(0, r) for r in range(8)}) == 8
