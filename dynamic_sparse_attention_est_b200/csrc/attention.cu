@@ -52,7 +52,10 @@ static_assert(128 * kRegsLoad + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "r
 // polynomial instead of MUFU ex2 (0 disables it).  Off by default: on B200 the
 // softmax is issue-bound rather than MUFU-bound (measured: dense 32K 7.97 ms
 // with 0, 8.41 ms with every 4th pair, 9.20 ms with every 2nd).
-constexpr int kEmuEvery = 4;
+#ifndef MINF_EMU_EVERY
+#define MINF_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = MINF_EMU_EVERY;
 
 enum : int {
     B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 4, B_V_FULL = 7, B_V_EMPTY = 10,
