@@ -45,8 +45,12 @@ constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment 
 // the load/MMA warpgroup drops to 56, the two softmax warpgroups rise to 224
 // (128 x 56 + 256 x 224 = 384 x 168).
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsLoad = 56;
-constexpr int kRegsSoftmax = 224;
+#ifndef MINF_REGS_LOAD
+#define MINF_REGS_LOAD 56
+#define MINF_REGS_SOFTMAX 224
+#endif
+constexpr int kRegsLoad = MINF_REGS_LOAD;
+constexpr int kRegsSoftmax = MINF_REGS_SOFTMAX;
 static_assert(128 * kRegsLoad + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 // Every kEmuEvery-th column pair takes its exponential from the FMA-pipe
 // polynomial instead of MUFU ex2 (0 disables it).  Off by default: on B200 the
