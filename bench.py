@@ -57,6 +57,26 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch, from the ncu capture summarised in profiles/, valid only for the
+# attention source it was taken on (sha1 of csrc/attention.cu).
+TRAFFIC = {
+    "vs-gqa-32k": ("38d73d8fa103efce0f7a33951b31e028137e348e", 5.383417e9 + 0.287480e9),
+}
+
+
+def attention_traffic(workload: str):
+    import hashlib
+
+    entry = TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    src = os.path.join(ROOT, "dynamic_sparse_attention_est_b200", "csrc", "attention.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha1(f.read()).hexdigest()
+    return entry[1] if sha == entry[0] else None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -384,7 +404,7 @@ def main():
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     achieved = tiles * TILE_FLOPS / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": attention_traffic(w.name),
                 "kernel": "attn_kernel (timed with its plan kernels, CUDA events around the attention call)",
                 "peak_source": f"{src} bf16_tflops_sustained"}
 
