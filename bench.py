@@ -197,6 +197,31 @@ def make_step(w, x, torch, minf, synth, seed):
     raise ValueError(w.pattern)
 
 
+def estimate_bytes(w) -> float:
+    """Algorithmic HBM bytes of one layer's index estimation (+ top-k), by pattern.
+
+    Vertical-Slash: both passes stream K once per pair of q-heads sharing a
+    kv-head (256 B per key), the vertical and slash score rows are written once
+    and read by five radix passes, the 191-offset diagonal partials are written
+    and read once.  Block-Sparse: Q and K are read once for pooling, the pooled
+    rows written, and the lower triangle of pooled scores written once and read
+    once by the per-row selection.
+    """
+    n, hq, hkv = w.n, w.hq, w.hkv
+    if w.pattern == "vs":
+        pairs = hkv * math.ceil((hq // hkv) / 2)
+        k_stream = 2 * pairs * n * 256
+        scores = 2 * hq * n * 4 * (1 + 5)
+        diag = 2 * hq * math.ceil(n / 128) * 191 * 4
+        return float(k_stream + scores + diag + hq * 64 * 256)
+    if w.pattern == "block":
+        nb = n // 64
+        pool = (hq + hkv) * n * 256 + (hq + hkv) * nb * 512
+        tri = hq * nb * (nb + 1) / 2 * 4
+        return float(pool + 2 * tri)
+    return 0.0
+
+
 def cpu_sample(w, x, orc, budget_s, seed):
     """Times the fp64 oracle on a bounded sample of the workload and scales it to one layer."""
     import numpy as np
@@ -430,6 +455,12 @@ def main():
             "roofline": roofline,
             "attention_ms": round(attn_ms, 4),
             "estimate_ms": round(ms_per_step - attn_ms, 4),
+            "estimate_roofline": ({"bound": "hbm", "bytes": estimate_bytes(w),
+                                   "achieved": round(estimate_bytes(w) / ((ms_per_step - attn_ms) * 1e-3) / 1e9, 1),
+                                   "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
+                                   "frac": round(estimate_bytes(w) / ((ms_per_step - attn_ms) * 1e-3) / 1e9
+                                                 / peaks.get("hbm_gbs"), 4)}
+                                  if w.pattern in ("vs", "block") and ms_per_step > attn_ms else None),
             "computed_tiles": tiles, "mask_pairs": pairs,
             "useful_tflops": round(4 * 128 * pairs / (attn_ms * 1e-3) / 1e12, 1),
             "dense": dense,

@@ -185,3 +185,90 @@ def test_bounded_wait_reports_timeout():
     out, _ = minf.minf_dense_attention(q, k, v)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
+
+
+# ----------------------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("n", [64, 192])
+def test_single_and_ragged_blocks_every_pattern(orc, n):
+    q, k, v = inputs(n, 2, 1, seed=n + 1)
+    qc, kc, vc = cuda(q, k, v)
+    ref, rl = orc.dense_attention(q, k, v, SCALE)
+    out, lse = minf.minf_dense_attention(qc, kc, vc, scale=SCALE)
+    check_attention(out, lse, ref, rl, f"dense n={n}")
+    ref, rl = orc.ashape_attention(q, k, v, SCALE, 16, 40)
+    out, lse = minf.minf_ashape_attention(qc, kc, vc, 16, 40, scale=SCALE)
+    check_attention(out, lse, ref, rl, f"A-shape n={n}")
+    bi, bc = orc.block_estimate(q, k, 64, 2)
+    gbi, gbc = minf.minf_block_estimate(qc, kc, topk=2)
+    assert np.array_equal(gbi.cpu().numpy(), bi) and np.array_equal(gbc.cpu().numpy(), bc)
+    ref, rl = orc.block_attention(q, k, v, SCALE, 64, bi, bc)
+    out, lse = minf.minf_block_attention(qc, kc, vc, gbi, gbc, scale=SCALE)
+    check_attention(out, lse, ref, rl, f"block n={n}")
+    vi, si, vert, slash = orc.vs_estimate(q, k, 64, 8, 16, SCALE, return_scores=True)
+    gv, gs = minf.minf_vs_estimate(qc, kc, 64, 8, 16, scale=SCALE)
+    for hp in range(2):
+        check_topk_band(gv[hp].cpu().numpy(), vert[hp], 8, f"vertical n={n}")
+        check_topk_band(gs[hp].cpu().numpy(), slash[hp], 16, f"slash n={n}")
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    out, lse = minf.minf_vs_attention(qc, kc, vc, torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out, lse, ref, rl, f"VS n={n}")
+
+
+def test_budgets_above_n_pad_and_cover_everything(orc):
+    n = 256
+    q, k, v = inputs(n, 2, 1, seed=21)
+    qc, kc, vc = cuda(q, k, v)
+    gv, gs = minf.minf_vs_estimate(qc, kc, 64, 300, 400, scale=SCALE)
+    gv, gs = gv.cpu().numpy(), gs.cpu().numpy()
+    assert np.array_equal(gv[:, :n], np.tile(np.arange(n), (2, 1))) and np.all(gv[:, n:] == -1)
+    assert np.array_equal(gs[:, :n], np.tile(np.arange(n), (2, 1))) and np.all(gs[:, n:] == -1)
+    out, lse = minf.minf_vs_attention(qc, kc, vc, torch.from_numpy(gv).cuda(), torch.from_numpy(gs).cuda(),
+                                      scale=SCALE)
+    ref, rl = orc.dense_attention(q, k, v, SCALE)
+    check_attention(out, lse, ref, rl, "VS full budgets = dense")
+    bi, bc = minf.minf_block_estimate(qc, kc, topk=9)  # topk above the 4 blocks
+    out, lse = minf.minf_block_attention(qc, kc, vc, bi, bc, scale=SCALE)
+    check_attention(out, lse, ref, rl, "BS full budgets = dense")
+
+
+def test_empty_key_sets_give_zero_and_minus_inf(orc):
+    n = 320
+    q, k, v = inputs(n, 2, 1, seed=4)
+    qc, kc, vc = cuda(q, k, v)
+    nb = n // 64
+    bi = torch.full((2, nb, 3), -1, dtype=torch.int32)
+    bc = torch.zeros(2, nb, dtype=torch.int32)
+    bi[0, 2, 0] = 1  # one query block of head 0 sees key block 1; everything else is empty
+    bc[0, 2] = 1
+    ref, rl = orc.block_attention(q, k, v, SCALE, 64, bi.numpy(), bc.numpy())
+    out, lse = minf.minf_block_attention(qc, kc, vc, bi.cuda(), bc.cuda(), scale=SCALE)
+    check_attention(out, lse, ref, rl, "block with empty rows")
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    vi = torch.full((2, 4), -1, dtype=torch.int32)
+    si = torch.full((2, 4), -1, dtype=torch.int32)
+    si[0, 0] = 0  # head 0: the main diagonal only (each query attends to itself)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi.numpy(), si.numpy())
+    out, lse = minf.minf_vs_attention(qc, kc, vc, vi.cuda(), si.cuda(), scale=SCALE)
+    check_attention(out, lse, ref, rl, "VS diagonal only / empty")
+    assert torch.equal(out[0], vc[0])  # softmax over one key returns that value row exactly
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+
+
+def test_many_heads_and_unsorted_head_subset(orc):
+    n, hq, hkv = 384, 16, 4
+    q, k, v = inputs(n, hq, hkv, seed=8)
+    ids = [15, 2, 7, 8, 3]
+    qc, kc, vc = cuda(q, k, v)
+    ref, rl = orc.ashape_attention(q, k, v, SCALE, 64, 100, head_ids=ids)
+    out, lse = minf.minf_ashape_attention(qc, kc, vc, 64, 100, scale=SCALE, head_ids=ids)
+    check_attention(out, lse, ref, rl, "A-shape head subset")
+    vi, si, vert, slash = orc.vs_estimate(q, k, 48, 20, 30, SCALE, head_ids=ids, return_scores=True)
+    gv, gs = minf.minf_vs_estimate(qc, kc, 48, 20, 30, scale=SCALE, head_ids=ids)
+    for p in range(len(ids)):
+        check_topk_band(gv[p].cpu().numpy(), vert[p], 20, f"vertical subset {p}")
+        check_topk_band(gs[p].cpu().numpy(), slash[p], 30, f"slash subset {p}")
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si, head_ids=ids)
+    out, lse = minf.minf_vs_attention(qc, kc, vc, torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE, head_ids=ids)
+    check_attention(out, lse, ref, rl, "VS head subset")
