@@ -6,6 +6,7 @@ A step is one pass of the whole path over one layer of synthetic input:
   vs-gqa-32k       minf_vs_estimate + minf_vs_attention (32 q-heads / 8 kv-heads, 32K tokens)
   block-gqa-128k   minf_block_estimate + minf_block_attention (128K tokens)
   ashape-gqa-128k  minf_ashape_attention (128K tokens)
+  trishape-gqa-128k minf_trishape_attention (A-shape + dense last 64 rows, 128K tokens)
   mixed-gqa-1m     minf_mixed_layer, per-head patterns drawn from the seed (1M tokens)
 The default is vs-gqa-32k.  Inputs stay resident in HBM and are larger than L2,
 so no flush is needed between steps.  The line also carries the roofline of the
@@ -183,6 +184,15 @@ def make_step(w, x, torch, minf, synth, seed):
             minf.minf_ashape_attention(q, k, v, w.n_sink, w.window, scale, out=out, want_lse=False, ws=ws)
 
         return (lambda: None), attend, ws, out, 0, 1
+    if w.pattern == "trishape":
+        ws = minf.workspace(256, dev)
+        out = torch.empty_like(q)
+
+        def attend():
+            minf.minf_trishape_attention(q, k, v, w.n_sink, w.window, w.last_q, scale, out=out, want_lse=False,
+                                         ws=ws)
+
+        return (lambda: None), attend, ws, out, 0, 1
     if w.pattern == "mixed":
         pats = synth.mixed_head_patterns(w, seed)
         ws = minf.workspace(minf.workspace_bytes(minf.OP_MIXED_LAYER, hq, hkv, n, hq, w.n_vertical, w.n_slash,
@@ -260,6 +270,8 @@ def cpu_sample(w, x, orc, budget_s, seed):
                 bi = np.tile(np.arange(w.topk, dtype=np.int32), (1, n // 64, 1))
                 bc = np.full((1, n // 64), w.topk, np.int32)
             orc.block_attention(q1, k1, v1, scale, 64, bi, bc, rows=rows)
+        elif w.pattern == "trishape":
+            orc.trishape_attention(q1, k1, v1, scale, w.n_sink, w.window, w.last_q, rows=rows)
         else:
             orc.ashape_attention(q1, k1, v1, scale, w.n_sink, w.window, rows=rows)
         dt = time.perf_counter() - t1

@@ -363,7 +363,7 @@ int do_block_attention(const Common &c, const void *q, const void *k, const void
 }
 
 int do_static_attention(int pattern, const Common &c, const void *q, const void *k, const void *v, float scale,
-                        int n_sink, int window, void *out, float *lse, void *ws, bool slot_is_id,
+                        int n_sink, int window, int n_last, void *out, float *lse, void *ws, bool slot_is_id,
                         cudaStream_t st) {
     AttnParams P;
     memset(&P, 0, sizeof(P));
@@ -372,6 +372,7 @@ int do_static_attention(int pattern, const Common &c, const void *q, const void 
     if (e != cudaSuccess) return cuda_fail(e, "tensor map");
     P.n_sink = n_sink;
     P.window = window;
+    P.n_last = n_last;
     e = run_attention(pattern, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "attention launch");
 }
@@ -442,6 +443,7 @@ size_t minf_workspace_bytes(int op, int hq, int hkv, int n, int n_heads, int p1,
         if (p1 < 1) return 0;
         return bytes_bs_attn(n, n_heads, p1);
     case MINF_OP_ASHAPE_ATTENTION:
+    case MINF_OP_TRISHAPE_ATTENTION:
     case MINF_OP_DENSE_ATTENTION:
         return MINF_STATUS_BYTES;
     case MINF_OP_MIXED_LAYER: {
@@ -543,7 +545,26 @@ int minf_ashape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf1
     if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
-    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, out, lse, ws, false,
+    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, 0, out, lse, ws, false,
+                               (cudaStream_t)stream);
+}
+
+int minf_trishape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n,
+                            int d, float scale, const int32_t *head_ids, int n_heads, int n_sink, int window,
+                            int n_last, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                            minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v || !out) return fail(MINF_ERR_INVALID, "null v or out");
+    if (!aligned16(v) || !aligned16(out)) return fail(MINF_ERR_INVALID, "v/out not 16-byte aligned");
+    if (n_sink < 0 || window < 1 || n_last < 0)
+        return fail(MINF_ERR_INVALID, "n_sink >= 0, window >= 1 and n_last >= 0 required");
+    if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
+    if ((rc = select_device(q))) return rc;
+    if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
+    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, n_last, out, lse, ws, false,
                                (cudaStream_t)stream);
 }
 
@@ -559,7 +580,7 @@ int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16
     if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
-    return do_static_attention(PAT_DENSE, c, q, k, v, scale, 0, 1, out, lse, ws, false, (cudaStream_t)stream);
+    return do_static_attention(PAT_DENSE, c, q, k, v, scale, 0, 1, 0, out, lse, ws, false, (cudaStream_t)stream);
 }
 
 int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
@@ -576,14 +597,14 @@ int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v,
         return fail(MINF_ERR_INVALID, "bad pattern parameters");
     if (last_q > 64) return fail(MINF_ERR_UNSUPPORTED, "last_q %d above 64", last_q);
     if (n / kBlock > 32768) return fail(MINF_ERR_UNSUPPORTED, "more than 32768 blocks");
-    Common sub[4];
-    for (int p = 0; p < 4; ++p) {
+    Common sub[5];
+    for (int p = 0; p < 5; ++p) {
         sub[p] = all;
         sub[p].n_heads = 0;
     }
     for (int h = 0; h < hq; ++h) {
         const int p = head_pattern[h];
-        if (p < 0 || p > 3) return fail(MINF_ERR_INVALID, "head %d: pattern code %d", h, p);
+        if (p < 0 || p > 4) return fail(MINF_ERR_INVALID, "head %d: pattern code %d", h, p);
         sub[p].ids[sub[p].n_heads++] = h;
     }
     const size_t need = minf_workspace_bytes(MINF_OP_MIXED_LAYER, hq, hkv, n, hq, n_vertical, n_slash, topk);
@@ -614,11 +635,17 @@ int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v,
         if (rc) return rc;
     }
     if (sub[PAT_ASHAPE].n_heads) {
-        rc = do_static_attention(PAT_ASHAPE, sub[PAT_ASHAPE], q, k, v, scale, n_sink, window, out, lse, ws, true, st);
+        rc = do_static_attention(PAT_ASHAPE, sub[PAT_ASHAPE], q, k, v, scale, n_sink, window, 0, out, lse, ws, true,
+                                 st);
+        if (rc) return rc;
+    }
+    if (sub[MINF_PATTERN_TRISHAPE].n_heads) {
+        rc = do_static_attention(PAT_ASHAPE, sub[MINF_PATTERN_TRISHAPE], q, k, v, scale, n_sink, window, last_q, out,
+                                 lse, ws, true, st);
         if (rc) return rc;
     }
     if (sub[PAT_DENSE].n_heads) {
-        rc = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, out, lse, ws, true, st);
+        rc = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, 0, out, lse, ws, true, st);
         if (rc) return rc;
     }
     return MINF_OK;

@@ -93,7 +93,8 @@ struct TileGen {
         } else if constexpr (PAT == PAT_ASHAPE) {
             sink_h = min((P.n_sink + kHalf - 1) / kHalf, nb64);
             w_lo = max(0, r0 - P.window + 1) / kHalf;
-            split = w_lo > sink_h;
+            // a tile holding dense tail rows (Tri-shape) needs every causal key
+            split = w_lo > sink_h && rmax < P.n - P.n_last;
             total = split ? sink_h + (hi - w_lo + 1) : hi + 1;
         } else if constexpr (PAT == PAT_BLOCK) {
             const int w = hp * P.n_qtiles + t;
@@ -132,7 +133,8 @@ struct TileGen {
             h.ks = blk * kHalf;
             h.len = kHalf;
             const bool full = (h.ks + kHalf - 1 <= r0) &&
-                              (h.ks + kHalf - 1 < P.n_sink || (r0 + kTileM - 1) - h.ks < P.window);
+                              (h.ks + kHalf - 1 < P.n_sink || (r0 + kTileM - 1) - h.ks < P.window ||
+                               r0 >= P.n - P.n_last);
             h.flags = HF_ROWS0 | HF_ROWS1 | (full ? HF_FULL : 0);
         } else if constexpr (PAT == PAT_BLOCK) {
             const int e = __ldg(plan + i);
@@ -190,7 +192,8 @@ __device__ __forceinline__ uint64_t half_mask(const AttnParams &P, const HalfDes
         const uint64_t sink = low_bits(P.n_sink - h.ks);
         const int c0 = q - h.ks - P.window + 1;  // first column inside the window
         const uint64_t win = c0 <= 0 ? ~0ull : (c0 >= 64 ? 0ull : (~0ull << c0));
-        return causal & (sink | win);
+        const uint64_t tail = q >= P.n - P.n_last ? ~0ull : 0ull;  // Tri-shape dense rows
+        return causal & (sink | win | tail);
     } else if constexpr (PAT == PAT_BLOCK) {
         const int half_row = r >> 6;
         return (h.flags & (HF_ROWS0 << half_row)) ? causal : 0ull;

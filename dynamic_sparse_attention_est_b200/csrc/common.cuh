@@ -52,8 +52,8 @@ struct AttnParams {
     int n, hq, hkv, group;
     int n_heads, n_qtiles;
     float scale_log2;
-    // A-shape
-    int n_sink, window;
+    // A-shape / Tri-shape (n_last > 0: the last n_last query rows attend densely)
+    int n_sink, window, n_last;
     // Block-Sparse plan: per work item (hp * n_qtiles + t), up to bs_stride half entries
     const int *bs_plan;
     const int *bs_cnt;

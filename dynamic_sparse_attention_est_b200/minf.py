@@ -34,8 +34,9 @@ OP_BLOCK_ATTENTION = 4
 OP_ASHAPE_ATTENTION = 5
 OP_DENSE_ATTENTION = 6
 OP_MIXED_LAYER = 7
+OP_TRISHAPE_ATTENTION = 8
 
-PATTERN_CODES = {"dense": 0, "vs": 1, "block": 2, "ashape": 3}
+PATTERN_CODES = {"dense": 0, "vs": 1, "block": 2, "ashape": 3, "trishape": 4}
 
 _P, _I, _F, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
 
@@ -46,6 +47,7 @@ _SIGS = {
     "minf_block_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_ashape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "minf_trishape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "minf_dense_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_mixed_layer": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "minf_vs_estimate_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P]),
@@ -230,6 +232,20 @@ def minf_ashape_attention(q, k, v, n_sink: int = 128, window: int = 4096, scale:
     _check(lib().minf_ashape_attention(_ptr(q), _ptr(k), _ptr(v), hq, hkv, n, d, _scale(scale), ids, nh, n_sink,
                                        window, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)),
            "minf_ashape_attention")
+    return out, lse
+
+
+def minf_trishape_attention(q, k, v, n_sink: int = 128, window: int = 4096, n_last: int = 64,
+                            scale: Optional[float] = None, head_ids=None, out=None, want_lse: bool = True, ws=None):
+    hq, hkv, n, d = _qkv(q, k, v)
+    ids, nh = _heads(hq, head_ids)
+    ws = _ws_for(ws, MINF_STATUS_BYTES, q.device)
+    out = torch.empty(nh, n, d, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty(nh, n, dtype=torch.float32, device=q.device) if want_lse else None
+    _check(lib().minf_trishape_attention(_ptr(q), _ptr(k), _ptr(v), hq, hkv, n, d, _scale(scale), ids, nh, n_sink,
+                                         window, n_last, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream(q.device)),
+           "minf_trishape_attention")
     return out, lse
 
 

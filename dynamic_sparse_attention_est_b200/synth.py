@@ -37,7 +37,7 @@ ROPE_THETA = 500000.0
 @dataclass(frozen=True)
 class Workload:
     name: str
-    pattern: str          # "vs", "block", "ashape", "dense" or "mixed"
+    pattern: str          # "vs", "block", "ashape", "trishape", "dense" or "mixed"
     hq: int
     hkv: int
     n: int
@@ -68,6 +68,8 @@ WORKLOADS: Dict[str, Workload] = {
                                 block=64, topk=100),
     "ashape-gqa-128k": Workload("ashape-gqa-128k", "ashape", 32, 8, 131072, "plain",
                                  n_sink=128, window=4096),
+    "trishape-gqa-128k": Workload("trishape-gqa-128k", "trishape", 32, 8, 131072, "plain",
+                                   n_sink=128, window=4096, last_q=64),
     # one Vertical-Slash head at 1M tokens with the layer's budgets: a profiling-size case
     "vs-1h-1m": Workload("vs-1h-1m", "vs", 1, 1, 1048576, "vertical", heavy_frac=0.005,
                           last_q=64, n_vertical=1000, n_slash=6096),

@@ -73,12 +73,14 @@ typedef struct CUstream_st *minf_stream_t; /* the same type as cudaStream_t */
 #define MINF_OP_ASHAPE_ATTENTION 5
 #define MINF_OP_DENSE_ATTENTION 6
 #define MINF_OP_MIXED_LAYER 7
+#define MINF_OP_TRISHAPE_ATTENTION 8
 
 /* Per-head pattern codes for minf_mixed_layer. */
 #define MINF_PATTERN_DENSE 0
 #define MINF_PATTERN_VS 1
 #define MINF_PATTERN_BLOCK 2
 #define MINF_PATTERN_ASHAPE 3
+#define MINF_PATTERN_TRISHAPE 4
 
 /*
  * Bytes of workspace an operation needs.  p1/p2/p3 by op:
@@ -155,6 +157,19 @@ int minf_ashape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf1
                           int n_heads, int n_sink, int window, minf_bf16 *out, float *lse,
                           void *ws, size_t ws_bytes, minf_stream_t stream);
 
+/*
+ * Tri-shape attention ([TALK], SCBench part: named as an A-shape variant that
+ * improves first-turn instruction following; the pages give no definition).
+ * This library's reading: the A-shape mask plus dense rows for the last n_last
+ * queries -- query i attends to key k iff k <= i and (k < n_sink or
+ * i - k < window or i >= n - n_last).  n_last = 0 is A-shape, n_last >= n is
+ * dense causal attention.
+ */
+int minf_trishape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
+                            int hkv, int n, int d, float scale, const int32_t *head_ids,
+                            int n_heads, int n_sink, int window, int n_last, minf_bf16 *out,
+                            float *lse, void *ws, size_t ws_bytes, minf_stream_t stream);
+
 /* Dense causal attention (the comparison baseline): query i attends to k <= i. */
 int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
                          int hkv, int n, int d, float scale, const int32_t *head_ids,
@@ -167,7 +182,9 @@ int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16
  * head_pattern is a HOST array of hq MINF_PATTERN_* codes.  VS heads run
  * minf_vs_estimate + minf_vs_attention (last_q, n_vertical, n_slash), BLOCK
  * heads minf_block_estimate + minf_block_attention (64, topk), ASHAPE heads
- * minf_ashape_attention (n_sink, window), DENSE heads minf_dense_attention.
+ * minf_ashape_attention (n_sink, window), TRISHAPE heads
+ * minf_trishape_attention (n_sink, window, n_last = last_q), DENSE heads
+ * minf_dense_attention.
  * out [hq][n][128] bf16, lse [hq][n] fp32 (nullable).  The indices are kept in
  * the workspace; everything runs on `stream`.
  */

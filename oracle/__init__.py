@@ -31,10 +31,11 @@ def build(mutant: int = 0, out_dir: Optional[str] = None, force: bool = False) -
     out = lib_path(mutant, out_dir)
     if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
         return out
+    tmp = f"{out}.{os.getpid()}.tmp"  # concurrent builders (spawned ranks) never share a temp file
     cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", f"-DORC_MUTANT={mutant}",
-           _SRC, "-o", out + ".tmp", "-lm"]
+           _SRC, "-o", tmp, "-lm"]
     subprocess.check_call(cmd)
-    os.replace(out + ".tmp", out)
+    os.replace(tmp, out)
     return out
 
 
@@ -47,6 +48,7 @@ _SIGS = {
     "orc_block_estimate": [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P],
     "orc_dense_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _P, _I, _P, _P],
     "orc_ashape_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _I, _P, _I, _P, _P],
+    "orc_trishape_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _I, _I, _P, _I, _P, _P],
     "orc_block_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P],
     "orc_vs_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P],
     "orc_threads": [],
@@ -162,6 +164,15 @@ class Oracle:
                                            d, scale, self._ptr(ids), nh, n_sink, window,
                                            self._ptr(r), nr, self._ptr(out), self._ptr(lse))
         self._check(rc, "ashape_attention")
+        return out, lse
+
+    def trishape_attention(self, q, k, v, scale: float, n_sink: int, window: int, n_last: int,
+                           head_ids=None, rows=None):
+        q, k, v, hq, hkv, n, d, ids, nh, r, nr, out, lse = self._attn_common(q, k, v, head_ids, rows)
+        rc = self.lib.orc_trishape_attention(self._ptr(q), self._ptr(k), self._ptr(v), hq, hkv, n,
+                                             d, scale, self._ptr(ids), nh, n_sink, window, n_last,
+                                             self._ptr(r), nr, self._ptr(out), self._ptr(lse))
+        self._check(rc, "trishape_attention")
         return out, lse
 
     def block_attention(self, q, k, v, scale: float, block: int, blk_idx, blk_cnt,

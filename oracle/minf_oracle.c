@@ -19,7 +19,9 @@
  *      `block` tokens, multiply the pooled matrices (mean pooling commutes with
  *      the matrix product), keep the top-k key blocks of each query block.
  *   3. A-shape ([TALK] second observation; [NEWS] 方法介绍): a static mask of the
- *      first tokens plus a local window.
+ *      first tokens plus a local window.  Tri-shape ([TALK], SCBench part, named
+ *      only as an A-shape variant): this build reads it as the A-shape mask plus
+ *      dense rows for the last queries.
  *   4. Masked-softmax attention over the key set each pattern selects, causal.
  *
  * Readings where the pages are silent (each is listed with its reason in the
@@ -241,11 +243,12 @@ static void attend_keys(const float *qi, const float *K, const float *V, int d, 
     *lse = m + log(den);
 }
 
-enum { PAT_DENSE = 0, PAT_ASHAPE = 1, PAT_BLOCK = 2, PAT_VS = 3 };
+enum { PAT_DENSE = 0, PAT_ASHAPE = 1, PAT_BLOCK = 2, PAT_VS = 3, PAT_TRISHAPE = 4 };
 
 typedef struct {
     int pattern;
-    int n_sink, window;                               /* A-shape */
+    int n_sink, window;                               /* A-shape, Tri-shape */
+    int n_last;                                       /* Tri-shape: dense last rows */
     const int *blk_idx, *blk_cnt; int topk, block;    /* Block-Sparse */
     const int *v_idx; int n_v; const int *s_idx; int n_s; /* Vertical-Slash */
 } mask_spec_t;
@@ -265,6 +268,15 @@ static int key_list(const mask_spec_t *ms, int hp, int i, int n, int *keys, unsi
             if (kk < ms->n_sink || i - kk < ms->window - 1) keys[nk++] = kk;
 #else
             if (kk < ms->n_sink || i - kk < ms->window) keys[nk++] = kk;
+#endif
+        break;
+    case PAT_TRISHAPE:
+        /* the A-shape lines, plus every key for the last n_last queries */
+        for (int kk = 0; kk <= i; ++kk)
+#if ORC_MUTANT == 7 /* planted: the dense tail one row short */
+            if (kk < ms->n_sink || i - kk < ms->window || i > n - ms->n_last) keys[nk++] = kk;
+#else
+            if (kk < ms->n_sink || i - kk < ms->window || i >= n - ms->n_last) keys[nk++] = kk;
 #endif
         break;
     case PAT_BLOCK: {
@@ -359,6 +371,22 @@ int orc_ashape_attention(const float *q, const float *k, const float *v, int hq,
     ms.pattern = PAT_ASHAPE;
     ms.n_sink = n_sink;
     ms.window = window;
+    return attend(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, &ms, rows, n_rows, out, lse);
+}
+
+/* Tri-shape: A-shape plus dense rows for the last n_last queries (the reading
+ * this build takes of the Tri-shape named in the AICon talk transcript
+ * "以 KV 缓存为中心的高效长文本方法", SCBench part, as an A-shape variant). */
+int orc_trishape_attention(const float *q, const float *k, const float *v, int hq, int hkv, int n,
+                           int d, double scale, const int *head_ids, int n_heads, int n_sink,
+                           int window, int n_last, const int *rows, int n_rows, double *out,
+                           double *lse) {
+    if (n_sink < 0 || window < 1 || n_last < 0) return ORC_ERR;
+    mask_spec_t ms = {0};
+    ms.pattern = PAT_TRISHAPE;
+    ms.n_sink = n_sink;
+    ms.window = window;
+    ms.n_last = n_last;
     return attend(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, &ms, rows, n_rows, out, lse);
 }
 

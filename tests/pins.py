@@ -224,6 +224,32 @@ def pin_attention_masks_bruteforce(orc):
             assert np.allclose(lse[hp], rl, rtol=1e-12), "A-shape lse"
 
 
+def _trishape_mask(n, sink, window, n_last):
+    i = np.arange(n)[:, None]
+    return _ashape_mask(n, sink, window) | ((np.arange(n)[None, :] <= i) & (i >= n - n_last))
+
+
+def pin_trishape_bruteforce(orc):
+    """Tri-shape: A-shape lines plus dense last rows, vs its dense-mask definition;
+    n_last = 0 is A-shape, n_last = n is dense."""
+    n = 256
+    scale = 1.0 / math.sqrt(128)
+    q, k, v, _ = _inputs(n, hq=2, hkv=1, seed=13)
+    f32 = lambda a: a.astype(np.float32)
+    for sink, window, n_last in [(16, 40, 64), (0, 1, 100), (5, 7, 1), (64, 300, 30)]:
+        out, lse = orc.trishape_attention(f32(q), f32(k), f32(v), scale, sink, window, n_last)
+        for hp in range(2):
+            ref, rl, _ = _masked_attention(q[hp], k[0], v[0], scale, _trishape_mask(n, sink, window, n_last))
+            assert np.allclose(out[hp], ref, rtol=1e-11, atol=1e-12), f"Tri-shape {sink}/{window}/{n_last}"
+            assert np.allclose(lse[hp], rl, rtol=1e-12), "Tri-shape lse"
+    a, _ = orc.ashape_attention(f32(q), f32(k), f32(v), scale, 16, 40)
+    t, _ = orc.trishape_attention(f32(q), f32(k), f32(v), scale, 16, 40, 0)
+    assert np.array_equal(a, t), "n_last = 0 is A-shape"
+    dns, _ = orc.dense_attention(f32(q), f32(k), f32(v), scale)
+    t, _ = orc.trishape_attention(f32(q), f32(k), f32(v), scale, 16, 40, n)
+    assert np.allclose(t, dns, rtol=1e-12, atol=1e-13), "n_last = n is dense"
+
+
 def pin_full_budget_is_dense(orc):
     """Budgets that cover every key reduce each pattern to dense causal attention."""
     n = 320
@@ -291,6 +317,7 @@ ALL_PINS = [
     pin_block_estimate_topk_bruteforce,
     pin_attention_masks_bruteforce,
     pin_full_budget_is_dense,
+    pin_trishape_bruteforce,
     pin_attention_closed_forms,
     pin_planted_recovery,
 ]

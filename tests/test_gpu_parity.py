@@ -272,3 +272,23 @@ def test_many_heads_and_unsorted_head_subset(orc):
     out, lse = minf.minf_vs_attention(qc, kc, vc, torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
                                       scale=SCALE, head_ids=ids)
     check_attention(out, lse, ref, rl, "VS head subset")
+
+
+@pytest.mark.parametrize("sink,window,n_last", [(128, 256, 64), (100, 300, 200), (0, 1, 1), (64, 64, 0), (7, 64, 5000)])
+def test_trishape(orc, sink, window, n_last):
+    n = 1344
+    q, k, v = inputs(n, 2, 1, structure="plain", seed=sink + window + n_last)
+    ref, rl = orc.trishape_attention(q, k, v, SCALE, sink, window, n_last)
+    out, lse = minf.minf_trishape_attention(*cuda(q, k, v), n_sink=sink, window=window, n_last=n_last, scale=SCALE)
+    check_attention(out, lse, ref, rl, f"Tri-shape {sink}/{window}/{n_last}")
+
+
+def test_mixed_layer_with_trishape(orc):
+    n, hq, hkv = 704, 4, 2
+    q, k, v = inputs(n, hq, hkv, seed=12)
+    pats = ["trishape", "vs", "trishape", "block"]
+    out, lse = minf.minf_mixed_layer(*cuda(q, k, v), pats, last_q=48, n_vertical=16, n_slash=32, topk=3,
+                                     n_sink=32, window=96, scale=SCALE)
+    for h in (0, 2):
+        ref, rl = orc.trishape_attention(q, k, v, SCALE, 32, 96, 48, head_ids=[h])
+        check_attention(out[h:h + 1], lse[h:h + 1], ref, rl, f"mixed Tri-shape head {h}")

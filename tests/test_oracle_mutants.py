@@ -17,6 +17,7 @@ MUTANTS = {
     4: "block diagonal not forced",
     5: "A-shape window one short",
     6: "VS key counted twice",
+    7: "Tri-shape dense tail one row short",
 }
 
 
