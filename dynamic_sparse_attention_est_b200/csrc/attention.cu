@@ -80,6 +80,7 @@ struct TileGen {
     const int *plan;
     // Vertical-Slash
     const int2 *groups;
+    const int *vl;  // this work item's gathered vertical keys, ascending
     int ng, gi, cur_a, cur_b, nsh, nvert;
 
     __device__ void init(const AttnParams &P, int hp, int t) {
@@ -109,6 +110,7 @@ struct TileGen {
             cur_b = 0;
             nsh = P.vs_nsh[w];
             nvert = P.vs_nvert[w];
+            vl = P.vs_vert + (size_t)w * P.vs_vstride;
             total = nsh + (nvert + kHalf - 1) / kHalf;
         }
     }
@@ -170,19 +172,42 @@ struct TileGen {
                 h.kind = HALF_GATHER;
                 h.ks = m * kHalf;
                 h.len = min(kHalf, nvert - m * kHalf);
-                h.flags = HF_ROWS0 | HF_ROWS1;
+                // every gathered key precedes the tile's first row: no element mask
+                const bool full = h.len == kHalf && __ldg(vl + h.ks + kHalf - 1) <= r0;
+                h.flags = HF_ROWS0 | HF_ROWS1 | (full ? HF_FULL : 0);
             }
         }
         return h;
     }
 };
 
+// Bitmap words a Vertical-Slash range half needs for one row; fetched one tile
+// ahead so that the loads' latency hides behind the current tile's softmax.
+struct MaskWords {
+    uint32_t s[3], v[3];
+};
+
+template <int PAT>
+__device__ __forceinline__ void mask_fetch(const AttnParams &P, const HalfDesc &h, int q,
+                                           const uint32_t *bits_s, const uint32_t *bits_v,
+                                           MaskWords &mw) {
+    if constexpr (PAT == PAT_VS) {
+        if (h.kind != HALF_RANGE) return;
+        const int ws0 = (q - h.ks - 63) >> 5, wv0 = h.ks >> 5;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const int a = ws0 + i, b = wv0 + i;
+            mw.s[i] = (a >= 0 && a < P.bit_words) ? __ldg(bits_s + a) : 0u;
+            mw.v[i] = (b >= 0 && b < P.bit_words) ? __ldg(bits_v + b) : 0u;
+        }
+    }
+}
+
 // Element mask of one half for query row q (= r0 + r): bit c set iff key c of
 // the half is inside the pattern's mask for q.
 template <int PAT>
 __device__ __forceinline__ uint64_t half_mask(const AttnParams &P, const HalfDesc &h, int q, int r,
-                                              const int *vlist, const uint32_t *bits_s,
-                                              const uint32_t *bits_v) {
+                                              const int *vlist, const MaskWords &mw) {
     if (h.kind == HALF_EMPTY) return 0ull;
     if (h.flags & HF_FULL) return ~0ull;
     const uint64_t causal = low_bits(q - h.ks + 1);
@@ -200,9 +225,12 @@ __device__ __forceinline__ uint64_t half_mask(const AttnParams &P, const HalfDes
     } else {
         const uint64_t lenm = low_bits(h.len);
         if (h.kind == HALF_RANGE) {
-            // slash: offset q - (ks + c) in S; vertical: key ks + c in V
-            const uint64_t ws = bits64_at(bits_s, P.bit_words, q - h.ks - 63);
-            const uint64_t wv = bits64_at(bits_v, P.bit_words, h.ks);
+            // slash: offset q - (ks + c) in S; vertical: key ks + c in V (words prefetched)
+            const int ss = (q - h.ks - 63) & 31, sv = h.ks & 31;
+            const uint64_t ws = (uint64_t)__funnelshift_r(mw.s[0], mw.s[1], ss) |
+                                ((uint64_t)__funnelshift_r(mw.s[1], mw.s[2], ss) << 32);
+            const uint64_t wv = (uint64_t)__funnelshift_r(mw.v[0], mw.v[1], sv) |
+                                ((uint64_t)__funnelshift_r(mw.v[1], mw.v[2], sv) << 32);
             return causal & lenm & (__brevll(ws) | wv);
         }
         // gathered verticals, ascending: keep those <= q
@@ -440,12 +468,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             gen.next(P);
             gen.next(P);
         }
+        HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
+        MaskWords mw0, mw1;
+        mask_fetch<PAT>(P, hd0, q, bits_s, bits_v, mw0);
+        mask_fetch<PAT>(P, hd1, q, bits_s, bits_v, mw1);
         for (int j = wg; j < T; j += 2) {
-            const HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
+            // the next own tile (j + 2): descriptors now, its mask words in flight meanwhile
             gen.next(P);  // the other warpgroup's tile j + 1
             gen.next(P);
-            const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, bits_s, bits_v);
-            const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, bits_s, bits_v);
+            const HalfDesc nd0 = gen.next(P), nd1 = gen.next(P);
+            MaskWords nw0, nw1;
+            mask_fetch<PAT>(P, nd0, q, bits_s, bits_v, nw0);
+            mask_fetch<PAT>(P, nd1, q, bits_s, bits_v, nw1);
+            const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, mw0);
+            const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, mw1);
             const bool full = (hd0.flags & hd1.flags & HF_FULL) != 0;  // uniform over the CTA
             if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
             const bool got = wait_bounded(bar(B_S_FULL + wg), (j >> 1) & 1, wc, wait_site(4 + wg, B_S_FULL + wg, j));
@@ -525,6 +561,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar(B_P_FULL + wg));
+            hd0 = nd0;
+            hd1 = nd1;
+            mw0 = nw0;
+            mw1 = nw1;
         }
         // ------------------------------------------------------------ epilogue
         ok = __all_sync(0xffffffffu, ok);
