@@ -75,6 +75,7 @@ VsEstBufs carve_vs_est(Carver &c, int n, int n_heads, int n_pairs) {
     b.diag = c.take<float>((size_t)n_heads * b.n_ktiles * 191);
     b.vert = c.take<float>((size_t)n_heads * n);
     b.slash = c.take<float>((size_t)n_heads * n);
+    b.topk_scratch = c.take<char>(topk_scratch_bytes(n_heads, n));
     return b;
 }
 

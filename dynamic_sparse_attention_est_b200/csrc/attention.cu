@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "topk.cuh"
 
 namespace minf {
 
@@ -692,63 +693,77 @@ __global__ void vs_mark_kernel(const int *v_idx, int n_vertical, const int *s_id
     }
 }
 
-// Ordered extraction of the set bits of a bitmap by one warp.
-__device__ int warp_extract_bits(const uint32_t *bm, int words, int *out, int cap, int lane) {
+// Ordered extraction of the set bits of a bitmap by the NT threads of a block:
+// each thread takes 8 consecutive words per sweep and a block scan gives its
+// output position.
+constexpr int kExtractThreads = 1024;
+
+template <int NT>
+__device__ int block_extract_bits(const uint32_t *bm, int words, int *out, int cap, TopkShared &sh) {
     int base = 0;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-        uint32_t word = (w0 + lane < words) ? bm[w0 + lane] : 0u;
-        const int c = __popc(word);
-        int incl = c;
+    for (int w0 = 0; w0 < words; w0 += NT * 8) {
+        const int wb = w0 + (int)threadIdx.x * 8;
+        uint32_t wd[8];
+        int c = 0;
 #pragma unroll
-        for (int s = 1; s < 32; s <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, s);
-            if (lane >= s) incl += y;
+        for (int e = 0; e < 8; ++e) {
+            wd[e] = (wb + e < words) ? bm[wb + e] : 0u;
+            c += __popc(wd[e]);
         }
-        int pos = base + incl - c;
-        while (word) {
-            const int b = __ffs(word) - 1;
-            if (pos < cap) out[pos] = (w0 + lane) * 32 + b;
-            ++pos;
-            word &= word - 1;
+        int tot;
+        int pos = base + block_excl_scan<NT>(c, &tot, sh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            uint32_t word = wd[e];
+            while (word) {
+                const int b = __ffs(word) - 1;
+                if (pos < cap) out[pos] = (wb + e) * 32 + b;
+                ++pos;
+                word &= word - 1;
+            }
         }
-        base += __shfl_sync(0xffffffffu, incl, 31);
+        base += tot;
     }
     return min(base, cap);
 }
 
 // Per head: sorted distinct verticals, and slash offsets merged into groups
-// whose 128-row key ranges touch (consecutive offsets at most 128 apart).
-__global__ void vs_extract_kernel(const uint32_t *bits_v, const uint32_t *bits_s, int words, int *vsorted,
-                                  int *nvs, int vcap, int *soff, int scap, int2 *groups, int *ngroups) {
-    const int hp = blockIdx.x, lane = threadIdx.x;
-    const int cv = warp_extract_bits(bits_v + (size_t)hp * words, words, vsorted + (size_t)hp * vcap, vcap, lane);
-    const int cs = warp_extract_bits(bits_s + (size_t)hp * words, words, soff + (size_t)hp * scap, scap, lane);
-    __syncwarp();
+// whose 128-row key ranges touch (consecutive offsets at most 128 apart).  A
+// group starts at an offset more than 128 past its predecessor and ends at
+// one more than 128 short of its successor; the j-th start and the j-th end
+// bound group j.
+__global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint32_t *bits_v, const uint32_t *bits_s,
+                                                                     int words, int *vsorted, int *nvs, int vcap,
+                                                                     int *soff, int scap, int2 *groups,
+                                                                     int *ngroups) {
+    __shared__ TopkShared sh;
+    const int hp = blockIdx.x;
+    const int cv = block_extract_bits<kExtractThreads>(bits_v + (size_t)hp * words, words,
+                                                       vsorted + (size_t)hp * vcap, vcap, sh);
+    const int cs = block_extract_bits<kExtractThreads>(bits_s + (size_t)hp * words, words,
+                                                       soff + (size_t)hp * scap, scap, sh);
+    __syncthreads();  // the offsets written above are read by other threads below
     const int *so = soff + (size_t)hp * scap;
     int2 *gr = groups + (size_t)hp * scap;
-    int ng = 0;
-    for (int e0 = 0; e0 < cs; e0 += 32) {
-        const int e = e0 + lane;
-        bool start = false;
-        if (e < cs) start = (e == 0) || (so[e] - so[e - 1] > kTileM);
-        const uint32_t bal = __ballot_sync(0xffffffffu, start);
-        if (start) gr[ng + __popc(bal & ((1u << lane) - 1u))].x = e;
-        ng += __popc(bal);
+    int n_start = 0, n_end = 0;
+    for (int e0 = 0; e0 < cs; e0 += kExtractThreads) {
+        const int e = e0 + (int)threadIdx.x;
+        int start = 0, end = 0, x = 0;
+        if (e < cs) {
+            x = so[e];
+            start = (e == 0) || (x - so[e - 1] > kTileM);
+            end = (e == cs - 1) || (so[e + 1] - x > kTileM);
+        }
+        int tot;
+        const int packed = block_excl_scan<kExtractThreads>(start | (end << 16), &tot, sh);
+        if (start) gr[n_start + (packed & 0xffff)].x = x;
+        if (end) gr[n_end + (packed >> 16)].y = x;
+        n_start += tot & 0xffff;
+        n_end += tot >> 16;
     }
-    __syncwarp();
-    for (int g0 = 0; g0 < ng; g0 += 32) {
-        const int gg = g0 + lane;
-        int s = gg < ng ? gr[gg].x : cs;
-        int nxt = __shfl_down_sync(0xffffffffu, s, 1);
-        if (lane == 31) nxt = (g0 + 32 < ng) ? gr[g0 + 32].x : cs;
-        if (gg >= ng - 1) nxt = cs;
-        __syncwarp();
-        if (gg < ng) gr[gg] = make_int2(so[s], so[nxt - 1]);
-        __syncwarp();
-    }
-    if (lane == 0) {
+    if (threadIdx.x == 0) {
         nvs[hp] = cv;
-        ngroups[hp] = ng;
+        ngroups[hp] = n_start;
     }
 }
 
@@ -870,7 +885,7 @@ cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, c
     if (e == cudaSuccess) e = cudaMemsetAsync(b.bits_s, 0, sizeof(uint32_t) * (size_t)n_heads * b.words, st);
     if (e != cudaSuccess) return e;
     vs_mark_kernel<<<n_heads, 256, 0, st>>>(v_idx, n_vertical, s_idx, n_slash, n, b.bits_v, b.bits_s, b.words);
-    vs_extract_kernel<<<n_heads, 32, 0, st>>>(b.bits_v, b.bits_s, b.words, b.vsorted, b.nvs, b.vcap, b.soff,
+    vs_extract_kernel<<<n_heads, kExtractThreads, 0, st>>>(b.bits_v, b.bits_s, b.words, b.vsorted, b.nvs, b.vcap, b.soff,
                                               b.scap, b.groups, b.ngroups);
     const int nw = n_heads * n_qtiles;
     vs_workitem_kernel<<<(nw + 3) / 4, 128, 0, st>>>(b.vsorted, b.nvs, b.vcap, b.groups, b.ngroups, b.scap,

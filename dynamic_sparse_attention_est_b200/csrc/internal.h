@@ -39,6 +39,7 @@ struct VsEstBufs {
     float *diag;    // [n_heads][n_ktiles][191] per key-tile diagonal partial sums
     float *vert;    // [n_heads][n]
     float *slash;   // [n_heads][n]
+    void *topk_scratch;  // topk_scratch_bytes(n_heads, n)
     int n_chunks, chunk_tiles, n_ktiles;
 };
 
@@ -80,6 +81,10 @@ cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaS
 
 // Top-k (largest first, ties to the lower index) of n_rows rows of `len`
 // non-negative floats each; writes min(k, len) indices ascending, -1 padded to k.
-cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, cudaStream_t st);
+// Rows longer than the one-block limit need topk_scratch_bytes(n_rows, len)
+// bytes of device scratch (256-byte aligned); shorter rows need none.
+size_t topk_scratch_bytes(int n_rows, int len);
+cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
+                          cudaStream_t st);
 
 }  // namespace minf

@@ -83,15 +83,33 @@ __device__ void block_topk_ascending(const float *x, int len, int k, int *out, i
             }
         }
         __syncthreads();
-        if (tid == 0) {
-            int cum = 0, d = 255;
-            for (; d > 0; --d) {
-                const int hcount = (int)sh.hist[d];
-                if (cum + hcount >= rem) break;
-                cum += hcount;
+        if (tid < 32) {
+            // lane L owns bins 255-8L .. 248-8L; a scan over lanes from the top
+            // finds the lane whose bins hold the rem-th largest key.
+            int c[8], sum = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                c[e] = (int)sh.hist[255 - 8 * tid - e];
+                sum += c[e];
             }
-            sh.digit = d;
-            sh.remaining = rem - cum;
+            int incl = sum;
+#pragma unroll
+            for (int s = 1; s < 32; s <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, s);
+                if (tid >= s) incl += y;
+            }
+            int cum = incl - sum;
+            if (cum < rem && incl >= rem) {
+                int d = 255 - 8 * tid;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (cum + c[e] >= rem) break;
+                    cum += c[e];
+                    --d;
+                }
+                sh.digit = d;
+                sh.remaining = rem - cum;
+            }
         }
         __syncthreads();
         prefix |= (uint32_t)sh.digit << shift;

@@ -321,9 +321,9 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
     slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, st);
+    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, b.topk_scratch, st);
     if (e != cudaSuccess) return e;
-    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, st);
+    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, b.topk_scratch, st);
 }
 
 }  // namespace minf

@@ -115,7 +115,8 @@ def test_vs_attention_unsorted_duplicate_indices(orc):
 
 
 @pytest.mark.parametrize("n,hq,hkv,last_q,nv,ns", [(4096, 1, 1, 64, 256, 512), (2048, 4, 2, 64, 100, 300),
-                                                   (1088, 3, 1, 17, 30, 40)])
+                                                   (1088, 3, 1, 17, 30, 40),
+                                                   (65600, 2, 1, 64, 1000, 2000)])  # rows split over blocks
 def test_vs_estimate_band(orc, n, hq, hkv, last_q, nv, ns):
     q, k, _ = inputs(n, hq, hkv, seed=n + hq)
     vi, si, vert, slash = orc.vs_estimate(q, k, last_q, nv, ns, SCALE, return_scores=True)
@@ -292,3 +293,43 @@ def test_mixed_layer_with_trishape(orc):
     for h in (0, 2):
         ref, rl = orc.trishape_attention(q, k, v, SCALE, 32, 96, 48, head_ids=[h])
         check_attention(out[h:h + 1], lse[h:h + 1], ref, rl, f"mixed Tri-shape head {h}")
+
+
+@pytest.mark.parametrize("n", [49216, 65600])
+def test_long_rows_budgets_above_n(n):
+    """Rows longer than one block's shared memory: budgets at or above n take every index, -1 padded."""
+    q, k, _ = inputs(n, 1, 1, seed=3)
+    gv, gs = minf.minf_vs_estimate(*cuda(q, k), last_q=64, n_vertical=n + 5, n_slash=n, scale=SCALE)
+    gv, gs = gv.cpu().numpy()[0], gs.cpu().numpy()[0]
+    assert np.array_equal(gv[:n], np.arange(n)) and np.all(gv[n:] == -1)
+    assert np.array_equal(gs, np.arange(n))
+
+
+@pytest.mark.parametrize("n,nv", [(4096, 1000), (65600, 20000)])
+def test_vertical_exact_ties_go_to_lower_index(orc, n, nv):
+    """q = 0 gives every query row a uniform causal softmax, so every key column that all
+    the last rows see has the same vertical score, summed in the same order: an exact tie
+    that the selection breaks towards the lower index (as the oracle does)."""
+    last_q = 64
+    q, k, _ = inputs(n, 1, 1, seed=9)
+    q = torch.zeros_like(q)
+    vi, _, vert, _ = orc.vs_estimate(q, k, last_q, nv, 16, SCALE, return_scores=True)
+    assert np.array_equal(vi[0], np.arange(nv))
+    gv, _ = minf.minf_vs_estimate(*cuda(q, k), last_q=last_q, n_vertical=nv, n_slash=16, scale=SCALE)
+    assert np.array_equal(gv.cpu().numpy()[0], np.arange(nv))
+
+
+def test_vs_attention_many_slash_groups(orc):
+    """More than a thousand separate slash groups (offsets 130 apart) with merged extras,
+    over 140K keys: the group list spans several extraction sweeps; sampled rows."""
+    n = 140096
+    q, k, v = inputs(n, 1, 1, seed=17)
+    offs = sorted(set([j * 130 for j in range(1078)] + [j * 130 + 60 for j in range(0, 1078, 7)]))
+    si = np.array([offs], np.int32)
+    rng = np.random.default_rng(4)
+    vi = np.sort(rng.choice(n, 64, replace=False)).astype(np.int32)[None, :]
+    rows = np.unique(np.concatenate([rng.integers(0, n, 200), np.arange(n - 64, n), [0, 127, 128, 140000]]))
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si, rows=rows)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out[:, rows], lse[:, rows], ref, rl, "VS many groups")
