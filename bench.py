@@ -62,7 +62,7 @@ def parse():
 # launch, from the ncu capture summarised in profiles/, valid only for the
 # attention source it was taken on (sha1 of csrc/attention.cu).
 TRAFFIC = {
-    "vs-gqa-32k": ("38d73d8fa103efce0f7a33951b31e028137e348e", 5.383417e9 + 0.287480e9),
+    "vs-gqa-32k": ("3cca896177f4967d9fc8cbe5f5bea358bca4d306", 3.521955e9 + 0.260125e9),
 }
 
 

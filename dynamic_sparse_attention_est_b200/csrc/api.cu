@@ -94,6 +94,7 @@ VsPlanBufs carve_vs_plan(Carver &c, int n, int n_heads, int n_vertical, int n_sl
     b.ngroups = c.take<int>(n_heads);
     b.nsh = c.take<int>(nw);
     b.nvert = c.take<int>(nw);
+    b.nle = c.take<int>(nw);
     b.vlist = c.take<int>(nw * b.vcap);
     return b;
 }
@@ -316,6 +317,7 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
     P.vs_vert = b.vlist;
     P.vs_nvert = b.nvert;
     P.vs_nsh = b.nsh;
+    P.vs_nle = b.nle;
     P.vs_vstride = b.vcap;
     P.vs_bits_s = b.bits_s;
     P.vs_bits_v = b.bits_v;

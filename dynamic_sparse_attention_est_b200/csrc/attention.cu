@@ -81,8 +81,8 @@ struct TileGen {
     const int *plan;
     // Vertical-Slash
     const int2 *groups;
-    const int *vl;  // this work item's gathered vertical keys, ascending
-    int ng, gi, cur_a, cur_b, nsh, nvert;
+    int2 gnext;     // groups[gi], loaded one group ahead
+    int ng, gi, cur_a, cur_b, nsh, nvert, nle;
 
     __device__ void init(const AttnParams &P, int hp, int t) {
         r0 = t * kTileM;
@@ -107,11 +107,12 @@ struct TileGen {
             groups = P.vs_groups + (size_t)hp * P.vs_gstride;
             ng = P.vs_ngroups[hp];
             gi = 0;
+            gnext = ng > 0 ? __ldg(groups) : make_int2(0, 0);
             cur_a = 1;
             cur_b = 0;
             nsh = P.vs_nsh[w];
             nvert = P.vs_nvert[w];
-            vl = P.vs_vert + (size_t)w * P.vs_vstride;
+            nle = P.vs_nle[w];
             total = nsh + (nvert + kHalf - 1) / kHalf;
         }
     }
@@ -150,8 +151,9 @@ struct TileGen {
             if (i < nsh) {
                 if (cur_a > cur_b) {
                     while (gi < ng) {
-                        const int2 g = __ldg(groups + gi);
+                        const int2 g = gnext;
                         ++gi;
+                        if (gi < ng) gnext = __ldg(groups + gi);  // in flight until the next group is needed
                         const int a = max(0, r0 - g.y);
                         const int b = min(r0 + kTileM - 1 - g.x, rmax);
                         if (b >= a) {
@@ -174,7 +176,7 @@ struct TileGen {
                 h.ks = m * kHalf;
                 h.len = min(kHalf, nvert - m * kHalf);
                 // every gathered key precedes the tile's first row: no element mask
-                const bool full = h.len == kHalf && __ldg(vl + h.ks + kHalf - 1) <= r0;
+                const bool full = h.len == kHalf && h.ks + kHalf <= nle;
                 h.flags = HF_ROWS0 | HF_ROWS1 | (full ? HF_FULL : 0);
             }
         }
@@ -777,11 +779,12 @@ __device__ __forceinline__ bool any_bits(const uint32_t *bm, int lo, int hi) {
     return false;
 }
 
-// Per work item (one warp): number of slash half-tiles, and the ascending list
-// of vertical keys that no slash range of this 128-row tile covers.
+// Per work item (one warp): number of slash half-tiles, the ascending list of
+// vertical keys that no slash range of this 128-row tile covers, and how many
+// of those precede the tile's first row (their halves need no element mask).
 __global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap, const int2 *groups,
                                    const int *ngroups, int gstride, const uint32_t *bits_s, int words, int n,
-                                   int n_heads, int n_qtiles, int *nsh, int *nvert, int *vlist) {
+                                   int n_heads, int n_qtiles, int *nsh, int *nvert, int *nle, int *vlist) {
     const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (w >= n_heads * n_qtiles) return;
@@ -801,7 +804,7 @@ __global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap,
     const uint32_t *bs = bits_s + (size_t)hp * words;
     int *dst = vlist + (size_t)w * vcap;
     const int cv = nvs[hp];
-    int out = 0;
+    int out = 0, le = 0;
     for (int e0 = 0; e0 < cv; e0 += 32) {
         const int e = e0 + lane;
         bool keep = false;
@@ -815,10 +818,12 @@ __global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap,
         const uint32_t bal = __ballot_sync(0xffffffffu, keep);
         if (keep) dst[out + __popc(bal & ((1u << lane) - 1u))] = vs[e];
         out += __popc(bal);
+        le += __popc(__ballot_sync(0xffffffffu, keep && vs[e] <= r0));
     }
     if (lane == 0) {
         nsh[w] = halves;
         nvert[w] = out;
+        nle[w] = le;
     }
 }
 
@@ -890,7 +895,7 @@ cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, c
     const int nw = n_heads * n_qtiles;
     vs_workitem_kernel<<<(nw + 3) / 4, 128, 0, st>>>(b.vsorted, b.nvs, b.vcap, b.groups, b.ngroups, b.scap,
                                                      b.bits_s, b.words, n, n_heads, n_qtiles, b.nsh, b.nvert,
-                                                     b.vlist);
+                                                     b.nle, b.vlist);
     return cudaGetLastError();
 }
 

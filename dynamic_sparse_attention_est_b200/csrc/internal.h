@@ -19,7 +19,7 @@ struct VsPlanBufs {
     int2 *groups;               // [n_heads][scap]
     int *ngroups;               // [n_heads]
     int scap;
-    int *nsh, *nvert;           // [n_work]
+    int *nsh, *nvert, *nle;     // [n_work]
     int *vlist;                 // [n_work][vcap]
 };
 

@@ -62,6 +62,16 @@ struct WaitCtl {
     uint64_t limit_ns;
 };
 
+// Records a wait that gave up: sets the CTA's abort flag and the status word.
+__device__ __forceinline__ void wait_gave_up(const WaitCtl &w, int site) {
+    *w.abort_flag = 1;
+    if (w.status) {
+        atomicExch(w.status, -4);
+        atomicCAS(w.status + 1, 0, site | 0x40000000);
+    }
+    __threadfence();
+}
+
 // `site` identifies the wait (role << 24 | barrier << 16 | tile) for diagnosis.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl &w, int site = 0) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -70,12 +80,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
         if (mbar_try_wait(bar, parity)) return true;
         if (*w.abort_flag) return false;
         if (globaltimer_ns() - t0 > w.limit_ns) {
-            *w.abort_flag = 1;
-            if (w.status) {
-                atomicExch(w.status, -4);
-                atomicCAS(w.status + 1, 0, site | 0x40000000);
-            }
-            __threadfence();
+            wait_gave_up(w, site);
             return false;
         }
     }
