@@ -51,6 +51,7 @@ _SIGS = {
     "orc_trishape_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _I, _I, _P, _I, _P, _P],
     "orc_block_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _P, _P, _I, _P, _I, _P, _P],
     "orc_vs_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P],
+    "orc_vs_tiles_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _P, _I, _P, _I, _I, _P, _I, _P, _P],
     "orc_threads": [],
     "orc_mutant": [],
 }
@@ -194,6 +195,18 @@ class Oracle:
                                        self._ptr(si), si.shape[-1], self._ptr(r), nr,
                                        self._ptr(out), self._ptr(lse))
         self._check(rc, "vs_attention")
+        return out, lse
+
+    def vs_tiles_attention(self, q, k, v, scale: float, v_idx, s_idx, tile_rows: int = 128,
+                           head_ids=None, rows=None):
+        """Vertical-Slash with whole slash tiles of ``tile_rows`` query rows."""
+        q, k, v, hq, hkv, n, d, ids, nh, r, nr, out, lse = self._attn_common(q, k, v, head_ids, rows)
+        vi, si = self._i32(v_idx), self._i32(s_idx)
+        rc = self.lib.orc_vs_tiles_attention(self._ptr(q), self._ptr(k), self._ptr(v), hq, hkv, n, d,
+                                             scale, self._ptr(ids), nh, self._ptr(vi), vi.shape[-1],
+                                             self._ptr(si), si.shape[-1], tile_rows, self._ptr(r), nr,
+                                             self._ptr(out), self._ptr(lse))
+        self._check(rc, "vs_tiles_attention")
         return out, lse
 
     def threads(self) -> int:

@@ -23,6 +23,10 @@
  *      only as an A-shape variant): this build reads it as the A-shape mask plus
  *      dense rows for the last queries.
  *   4. Masked-softmax attention over the key set each pattern selects, causal.
+ *      Vertical-Slash has two key sets: token-exact (a key enters row i if it
+ *      is a vertical or i - k is a selected offset) and whole slash tiles
+ *      ([NEWS] Figure 4 computes slashes as dense blocks: every key an offset
+ *      reaches from some row of the query tile is attended by all its rows).
  *
  * Readings where the pages are silent (each is listed with its reason in the
  * design notes): logits are scale * q.k, softmax over keys k <= i (causal) in the
@@ -243,7 +247,7 @@ static void attend_keys(const float *qi, const float *K, const float *V, int d, 
     *lse = m + log(den);
 }
 
-enum { PAT_DENSE = 0, PAT_ASHAPE = 1, PAT_BLOCK = 2, PAT_VS = 3, PAT_TRISHAPE = 4 };
+enum { PAT_DENSE = 0, PAT_ASHAPE = 1, PAT_BLOCK = 2, PAT_VS = 3, PAT_TRISHAPE = 4, PAT_VS_TILES = 5 };
 
 typedef struct {
     int pattern;
@@ -251,6 +255,7 @@ typedef struct {
     int n_last;                                       /* Tri-shape: dense last rows */
     const int *blk_idx, *blk_cnt; int topk, block;    /* Block-Sparse */
     const int *v_idx; int n_v; const int *s_idx; int n_s; /* Vertical-Slash */
+    int tile_rows;                                    /* Vertical-Slash, whole slash tiles */
 } mask_spec_t;
 
 /* Builds the key list of query row i of head position hp, ascending, each key
@@ -312,6 +317,30 @@ static int key_list(const mask_spec_t *ms, int hp, int i, int n, int *keys, unsi
 #endif
                 mark[kk] = 0;
             }
+        break;
+    }
+    case PAT_VS_TILES: {
+        /* Slash ranges attended whole: row i of the tile_rows-row query tile that
+         * starts at r0 takes, for every selected offset o, the keys r0 - o ..
+         * r0 + tile_rows - 1 - o (the keys that o reaches from any row of its
+         * tile), plus the verticals; then only the causal bound k <= i. */
+        const int *vr = ms->v_idx + (size_t)hp * ms->n_v, *sr = ms->s_idx + (size_t)hp * ms->n_s;
+        const int r0 = i - i % ms->tile_rows;
+#if ORC_MUTANT == 8 /* planted: the range one key too wide */
+        const int span = ms->tile_rows;
+#else
+        const int span = ms->tile_rows - 1;
+#endif
+        for (int j = 0; j < ms->n_v; ++j)
+            if (vr[j] >= 0 && vr[j] <= i) mark[vr[j]] = 1;
+        for (int j = 0; j < ms->n_s; ++j) {
+            const int o = sr[j];
+            if (o < 0 || o >= n) continue;
+            const int lo = r0 - o < 0 ? 0 : r0 - o, hi = r0 + span - o < i ? r0 + span - o : i;
+            for (int kk = lo; kk <= hi; ++kk) mark[kk] = 1;
+        }
+        for (int kk = 0; kk <= i; ++kk)
+            if (mark[kk]) { keys[nk++] = kk; mark[kk] = 0; }
         break;
     }
     }
@@ -415,6 +444,24 @@ int orc_vs_attention(const float *q, const float *k, const float *v, int hq, int
     ms.n_v = n_vertical;
     ms.s_idx = s_idx;
     ms.n_s = n_slash;
+    return attend(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, &ms, rows, n_rows, out, lse);
+}
+
+/* Vertical-Slash with every computed slash range attended whole by the rows of
+ * its query tile (the pages' kernel computes slashes as dense blocks: news
+ * article "单卡A100实现百万token推理…", Figure 4); tile_rows is the query tile height. */
+int orc_vs_tiles_attention(const float *q, const float *k, const float *v, int hq, int hkv, int n,
+                           int d, double scale, const int *head_ids, int n_heads, const int *v_idx,
+                           int n_vertical, const int *s_idx, int n_slash, int tile_rows,
+                           const int *rows, int n_rows, double *out, double *lse) {
+    if (!v_idx || !s_idx || n_vertical <= 0 || n_slash <= 0 || tile_rows <= 0) return ORC_ERR;
+    mask_spec_t ms = {0};
+    ms.pattern = PAT_VS_TILES;
+    ms.v_idx = v_idx;
+    ms.n_v = n_vertical;
+    ms.s_idx = s_idx;
+    ms.n_s = n_slash;
+    ms.tile_rows = tile_rows;
     return attend(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, &ms, rows, n_rows, out, lse);
 }
 

@@ -250,6 +250,57 @@ def pin_trishape_bruteforce(orc):
     assert np.allclose(t, dns, rtol=1e-12, atol=1e-13), "n_last = n is dense"
 
 
+def pin_vs_tiles_forms(orc):
+    """Vertical-Slash with whole slash tiles ([NEWS] Figure 4: slashes computed as
+    dense blocks), against forms that follow from its definition:
+      * offset 0 alone: row i attends its tile's causal prefix, keys r0 .. i;
+      * one offset o >= tile: every row of the tile starting at r0 attends exactly
+        the tile_rows keys r0 - o .. r0 + tile_rows - 1 - o (none for the first
+        tiles, which then give o = 0 and lse = -inf);
+      * tile_rows = 1 is the token-exact pattern;
+      * the token-exact key set is a subset: lse can only grow;
+      * every offset selected is dense attention."""
+    n, T = 320, 128
+    scale = 1.0 / math.sqrt(128)
+    q, k, v, _ = _inputs(n, hq=2, hkv=1, seed=23)
+    f32 = lambda a: a.astype(np.float32)
+    i = np.arange(n)[:, None]
+    kk = np.arange(n)[None, :]
+    r0 = (i // T) * T
+    none_v = np.full((2, 1), -1, np.int32)
+    out, lse = orc.vs_tiles_attention(f32(q), f32(k), f32(v), scale, none_v, np.zeros((2, 1), np.int32), T)
+    for hp in range(2):
+        ref, rl, _ = _masked_attention(q[hp], k[0], v[0], scale, (kk >= r0) & (kk <= i))
+        assert np.allclose(out[hp], ref, rtol=1e-11, atol=1e-12), "offset 0: tile prefix"
+        assert np.allclose(lse[hp], rl, rtol=1e-12), "offset 0: lse"
+    o = 200
+    out, lse = orc.vs_tiles_attention(f32(q), f32(k), f32(v), scale, none_v, np.full((2, 1), o, np.int32), T)
+    for hp in range(2):
+        mask = (kk >= r0 - o) & (kk < r0 - o + T) & (kk >= 0)
+        ref, rl, _ = _masked_attention(q[hp], k[0], v[0], scale, mask)
+        assert np.allclose(out[hp], ref, rtol=1e-11, atol=1e-12), "one far offset: a fixed key range per tile"
+        assert np.array_equal(np.isfinite(lse[hp]), np.isfinite(rl)), "empty rows"
+        fin = np.isfinite(rl)
+        assert np.allclose(lse[hp][fin], rl[fin], rtol=1e-12), "one far offset: lse"
+        counts = mask.sum(axis=1)
+        assert set(np.unique(counts[i[:, 0] >= 2 * T]).tolist()) == {T}, "tile_rows keys per row"
+    rng = np.random.default_rng(29)
+    vi = np.sort(rng.choice(n, (2, 12), replace=False), axis=1).astype(np.int32)
+    si = np.concatenate([np.zeros((2, 1), np.int32),
+                         np.sort(rng.choice(np.arange(1, n), (2, 15), replace=False), axis=1)], axis=1).astype(np.int32)
+    exact, el = orc.vs_attention(f32(q), f32(k), f32(v), scale, vi, si)
+    one, ol = orc.vs_tiles_attention(f32(q), f32(k), f32(v), scale, vi, si, 1)
+    assert np.allclose(one, exact, rtol=1e-12, atol=1e-13) and np.allclose(ol, el, rtol=1e-12), \
+        "tile_rows = 1 is token-exact"
+    _, tl = orc.vs_tiles_attention(f32(q), f32(k), f32(v), scale, vi, si, T)
+    assert np.all(tl >= el - 1e-12), "whole tiles attend a superset"
+    assert np.any(tl > el + 1e-6), "and strictly more somewhere"
+    dense, _ = orc.dense_attention(f32(q), f32(k), f32(v), scale)
+    all_o = np.tile(np.arange(n, dtype=np.int32), (2, 1))
+    out, _ = orc.vs_tiles_attention(f32(q), f32(k), f32(v), scale, none_v, all_o, T)
+    assert np.allclose(out, dense, rtol=1e-12, atol=1e-13), "every offset: dense"
+
+
 def pin_full_budget_is_dense(orc):
     """Budgets that cover every key reduce each pattern to dense causal attention."""
     n = 320
@@ -318,6 +369,7 @@ ALL_PINS = [
     pin_attention_masks_bruteforce,
     pin_full_budget_is_dense,
     pin_trishape_bruteforce,
+    pin_vs_tiles_forms,
     pin_attention_closed_forms,
     pin_planted_recovery,
 ]
