@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--workload", default="vs-gqa-32k")
     ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--vs-mode", default="exact", choices=["exact", "tiles"],
+                    help="Vertical-Slash key set: token-exact, or every computed slash range attended whole")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-kernel comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work to sample")
@@ -69,7 +71,7 @@ TRAFFIC = {
 def attention_traffic(workload: str):
     import hashlib
 
-    entry = TRAFFIC.get(workload)
+    entry = TRAFFIC.get(workload) if workload else None
     if entry is None:
         return None
     src = os.path.join(ROOT, "dynamic_sparse_attention_est_b200", "csrc", "attention.cu")
@@ -140,7 +142,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workload
-def make_step(w, x, torch, minf, synth, seed):
+def make_step(w, x, torch, minf, synth, seed, vs_mode="exact"):
     """Returns (step(ws) -> out, attention-only call for timing, label of the attention call)."""
     q, k, v = x["q"], x["k"], x["v"]
     hq, hkv, n = w.hq, w.hkv, w.n
@@ -156,9 +158,11 @@ def make_step(w, x, torch, minf, synth, seed):
         def estimate():
             state["idx"] = minf.minf_vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, scale, ws=ws_est)
 
+        vs_attention = minf.minf_vs_attention_tiles if vs_mode == "tiles" else minf.minf_vs_attention
+
         def attend():
             vi, si = state["idx"]
-            minf.minf_vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
+            vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
 
         return estimate, attend, ws, out, 6, 4
     if w.pattern == "block":
@@ -232,7 +236,7 @@ def estimate_bytes(w) -> float:
     return 0.0
 
 
-def cpu_sample(w, x, orc, budget_s, seed):
+def cpu_sample(w, x, orc, budget_s, seed, vs_mode="exact"):
     """Times the fp64 oracle on a bounded sample of the workload and scales it to one layer."""
     import numpy as np
     import torch
@@ -263,7 +267,9 @@ def cpu_sample(w, x, orc, budget_s, seed):
     while True:
         rows = np.linspace(0, n - 1, nrows).astype(np.int32)
         t1 = time.perf_counter()
-        if w.pattern in ("vs", "mixed"):
+        if w.pattern == "vs" and vs_mode == "tiles":
+            orc.vs_tiles_attention(q1, k1, v1, scale, vi, si, 128, rows=rows)
+        elif w.pattern in ("vs", "mixed"):
             orc.vs_attention(q1, k1, v1, scale, vi, si, rows=rows)
         elif w.pattern == "block":
             if n // 64 > 4096:
@@ -309,14 +315,15 @@ def main():
         per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
         vals = []
         for i in range(args.warmup + args.steps):
-            r = cpu_sample(w, x, orc, per, args.seed)
+            r = cpu_sample(w, x, orc, per, args.seed, args.vs_mode)
             if i >= args.warmup:
                 vals.append(r["value"])
         val = statistics.median(vals)
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "hq": w.hq, "hkv": w.hkv, "n": w.n},
+                "config": {"workload": w.name, "hq": w.hq, "hkv": w.hkv, "n": w.n,
+                           **({"vs_mode": args.vs_mode} if w.pattern == "vs" else {})},
                 "cpu_baseline": {"value": val, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
                                  "sample": r["sample"]},
                 "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -341,7 +348,7 @@ def main():
     x = synth.generate(w, seed=seed, device=dev)
     torch.cuda.synchronize()
     log("inputs ready")
-    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed)
+    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed, args.vs_mode)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -396,7 +403,7 @@ def main():
         host_in = {key: x[key].cpu().pin_memory() for key in ("q", "k", "v")}
         x2 = {key: torch.empty_like(x[key]) for key in ("q", "k", "v")}
         sets = [(x, estimate, attend, out)]
-        e2, a2, _, o2, _, _ = make_step(w, x2, torch, minf, synth, seed)
+        e2, a2, _, o2, _, _ = make_step(w, x2, torch, minf, synth, seed, args.vs_mode)
         sets.append((x2, e2, a2, o2))
         host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -468,7 +475,7 @@ def main():
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     achieved = tiles * TILE_FLOPS / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": attention_traffic(w.name),
+                "frac": round(achieved / peak, 4), "traffic": attention_traffic(w.name if args.vs_mode == "exact" else None),
                 "kernel": "attn_kernel (timed with its plan kernels, CUDA events around the attention call)",
                 "peak_source": f"{src} bf16_tflops_sustained"}
 
@@ -478,7 +485,7 @@ def main():
         import oracle
 
         xs = {"q": x["q"][:1].cpu(), "k": x["k"][:1].cpu(), "v": x["v"][:1].cpu()}
-        cpu = cpu_sample(w, xs, oracle.get(), args.cpu_budget, seed)
+        cpu = cpu_sample(w, xs, oracle.get(), args.cpu_budget, seed, args.vs_mode)
 
     if rank == 0:
         line = {
@@ -489,6 +496,7 @@ def main():
             "config": {"workload": w.name, "pattern": w.pattern, "hq": w.hq, "hkv": w.hkv, "n": w.n,
                        "last_q": w.last_q, "n_vertical": w.n_vertical, "n_slash": w.n_slash, "topk": w.topk,
                        "n_sink": w.n_sink, "window": w.window,
+                       **({"vs_mode": args.vs_mode} if w.pattern == "vs" else {}),
                        "l2": "inputs larger than L2 (no flush)",
                        "parallelism": f"one layer per rank x{world}"},
             "roofline": roofline,

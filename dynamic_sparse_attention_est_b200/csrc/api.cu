@@ -301,7 +301,7 @@ int do_vs_estimate(const Common &c, const void *q, const void *k, int last_q, in
 
 int do_vs_attention(const Common &c, const void *q, const void *k, const void *v, float scale, const int32_t *v_idx,
                     int nv, const int32_t *s_idx, int ns, void *out, float *lse, void *ws, char *scratch,
-                    bool slot_is_id, cudaStream_t st) {
+                    bool slot_is_id, cudaStream_t st, bool tiles = false) {
     Carver cv(scratch, 0);
     VsPlanBufs b = carve_vs_plan(cv, c.n, c.n_heads, nv, ns);
     cudaError_t e = run_vs_plan(b, v_idx, nv, s_idx, ns, c.n, c.n_heads, qtiles(c.n), st);
@@ -322,6 +322,7 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
     P.vs_bits_s = b.bits_s;
     P.vs_bits_v = b.bits_v;
     P.bit_words = b.words;
+    P.vs_tiles = tiles ? 1 : 0;
     e = run_attention(PAT_VS, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "vs attention launch");
 }
@@ -483,10 +484,11 @@ int minf_vs_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, in
                           static_cast<char *>(ws) + MINF_STATUS_BYTES, (cudaStream_t)stream);
 }
 
-int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
-                      float scale, const int32_t *head_ids, int n_heads, const int32_t *v_idx, int n_vertical,
-                      const int32_t *s_idx, int n_slash, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
-                      minf_stream_t stream) {
+static int vs_attention_entry(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv,
+                              int n, int d, float scale, const int32_t *head_ids, int n_heads,
+                              const int32_t *v_idx, int n_vertical, const int32_t *s_idx, int n_slash,
+                              minf_bf16 *out, float *lse, void *ws, size_t ws_bytes, minf_stream_t stream,
+                              bool tiles) {
     Common c;
     int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
     if (rc) return rc;
@@ -498,7 +500,23 @@ int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
     return do_vs_attention(c, q, k, v, scale, v_idx, n_vertical, s_idx, n_slash, out, lse, ws,
-                           static_cast<char *>(ws) + MINF_STATUS_BYTES, false, (cudaStream_t)stream);
+                           static_cast<char *>(ws) + MINF_STATUS_BYTES, false, (cudaStream_t)stream, tiles);
+}
+
+int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
+                      float scale, const int32_t *head_ids, int n_heads, const int32_t *v_idx, int n_vertical,
+                      const int32_t *s_idx, int n_slash, minf_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                      minf_stream_t stream) {
+    return vs_attention_entry(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, v_idx, n_vertical, s_idx, n_slash,
+                              out, lse, ws, ws_bytes, stream, false);
+}
+
+int minf_vs_attention_tiles(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n,
+                            int d, float scale, const int32_t *head_ids, int n_heads, const int32_t *v_idx,
+                            int n_vertical, const int32_t *s_idx, int n_slash, minf_bf16 *out, float *lse, void *ws,
+                            size_t ws_bytes, minf_stream_t stream) {
+    return vs_attention_entry(q, k, v, hq, hkv, n, d, scale, head_ids, n_heads, v_idx, n_vertical, s_idx, n_slash,
+                              out, lse, ws, ws_bytes, stream, true);
 }
 
 int minf_block_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d, int block, int topk,

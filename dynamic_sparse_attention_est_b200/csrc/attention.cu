@@ -167,7 +167,9 @@ struct TileGen {
                     h.kind = HALF_RANGE;
                     h.ks = cur_a;
                     h.len = min(kHalf, cur_b - cur_a + 1);
-                    h.flags = HF_ROWS0 | HF_ROWS1;
+                    // whole slash tiles: a full half below the tile's first row needs no mask
+                    const bool full = P.vs_tiles && h.len == kHalf && h.ks + kHalf - 1 <= r0;
+                    h.flags = HF_ROWS0 | HF_ROWS1 | (full ? HF_FULL : 0);
                     cur_a += kHalf;
                 }
             } else {
@@ -195,7 +197,7 @@ __device__ __forceinline__ void mask_fetch(const AttnParams &P, const HalfDesc &
                                            const uint32_t *bits_s, const uint32_t *bits_v,
                                            MaskWords &mw) {
     if constexpr (PAT == PAT_VS) {
-        if (h.kind != HALF_RANGE) return;
+        if (h.kind != HALF_RANGE || P.vs_tiles) return;
         const int ws0 = (q - h.ks - 63) >> 5, wv0 = h.ks >> 5;
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
@@ -227,6 +229,7 @@ __device__ __forceinline__ uint64_t half_mask(const AttnParams &P, const HalfDes
         return (h.flags & (HF_ROWS0 << half_row)) ? causal : 0ull;
     } else {
         const uint64_t lenm = low_bits(h.len);
+        if (h.kind == HALF_RANGE && P.vs_tiles) return causal & lenm;  // whole slash tiles
         if (h.kind == HALF_RANGE) {
             // slash: offset q - (ks + c) in S; vertical: key ks + c in V (words prefetched)
             const int ss = (q - h.ks - 63) & 31, sv = h.ks & 31;

@@ -66,6 +66,7 @@ struct AttnParams {
     const int *vs_nvert;      // per work item
     const int *vs_nsh;        // per work item: number of slash half-tiles
     const int *vs_nle;        // per work item: gathered keys at or before the tile's first row
+    int vs_tiles;             // 1: slash ranges attended whole (causal mask only)
     int vs_vstride;
     const uint32_t *vs_bits_s;  // per head: bitmap of slash offsets
     const uint32_t *vs_bits_v;  // per head: bitmap of vertical keys

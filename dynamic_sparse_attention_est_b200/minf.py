@@ -44,6 +44,7 @@ _SIGS = {
     "minf_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "minf_vs_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_vs_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "minf_vs_attention_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_ashape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -173,8 +174,7 @@ def minf_vs_estimate_noalloc(q, k, last_q: int = 64, n_vertical: int = 1000, n_s
     return v_idx, s_idx
 
 
-def minf_vs_attention(q, k, v, v_idx, s_idx, scale: Optional[float] = None, head_ids=None, out=None,
-                      want_lse: bool = True, ws=None):
+def _vs_attention(fn_name, q, k, v, v_idx, s_idx, scale, head_ids, out, want_lse, ws):
     hq, hkv, n, d = _qkv(q, k, v)
     ids, nh = _heads(hq, head_ids)
     v_idx = v_idx.to(torch.int32).contiguous()
@@ -183,11 +183,22 @@ def minf_vs_attention(q, k, v, v_idx, s_idx, scale: Optional[float] = None, head
     ws = _ws_for(ws, need, q.device)
     out = torch.empty(nh, n, d, dtype=torch.bfloat16, device=q.device) if out is None else out
     lse = torch.empty(nh, n, dtype=torch.float32, device=q.device) if want_lse else None
-    _check(lib().minf_vs_attention(_ptr(q), _ptr(k), _ptr(v), hq, hkv, n, d, _scale(scale), ids, nh, _ptr(v_idx),
+    _check(getattr(lib(), fn_name)(_ptr(q), _ptr(k), _ptr(v), hq, hkv, n, d, _scale(scale), ids, nh, _ptr(v_idx),
                                    v_idx.shape[-1], _ptr(s_idx), s_idx.shape[-1], _ptr(out), _ptr(lse), _ptr(ws),
                                    ws.numel(), _stream(q.device)),
-           "minf_vs_attention")
+           fn_name)
     return out, lse
+
+
+def minf_vs_attention(q, k, v, v_idx, s_idx, scale: Optional[float] = None, head_ids=None, out=None,
+                      want_lse: bool = True, ws=None):
+    return _vs_attention("minf_vs_attention", q, k, v, v_idx, s_idx, scale, head_ids, out, want_lse, ws)
+
+
+def minf_vs_attention_tiles(q, k, v, v_idx, s_idx, scale: Optional[float] = None, head_ids=None, out=None,
+                            want_lse: bool = True, ws=None):
+    """Vertical-Slash attention with every computed slash range attended whole."""
+    return _vs_attention("minf_vs_attention_tiles", q, k, v, v_idx, s_idx, scale, head_ids, out, want_lse, ws)
 
 
 def minf_block_estimate(q, k, topk: int = 100, block: int = 64, head_ids=None, ws=None):

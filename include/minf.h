@@ -123,6 +123,22 @@ int minf_vs_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v
                       minf_stream_t stream);
 
 /*
+ * Vertical-Slash sparse attention with whole slash tiles ([NEWS] Figure 4:
+ * slashes are computed as dense blocks).  Query i, in the 128-query tile that
+ * starts at r0 = i - i % 128, attends to key k iff k <= i and (k is in
+ * v_idx[p], or r0 - o <= k <= r0 + 127 - o for some offset o in s_idx[p]):
+ * every key a selected offset reaches from some row of the tile is attended by
+ * all its rows.  A superset of minf_vs_attention's key set, with no element
+ * mask inside the slash ranges.  Arguments, layouts, workspace
+ * (MINF_OP_VS_ATTENTION) and errors as minf_vs_attention.
+ */
+int minf_vs_attention_tiles(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq,
+                            int hkv, int n, int d, float scale, const int32_t *head_ids,
+                            int n_heads, const int32_t *v_idx, int n_vertical,
+                            const int32_t *s_idx, int n_slash, minf_bf16 *out, float *lse,
+                            void *ws, size_t ws_bytes, minf_stream_t stream);
+
+/*
  * Block-Sparse index estimation ([NEWS] 方法介绍).  Q and K are mean-pooled
  * over blocks of `block` (= 64) tokens in fp32; for query block i the pooled
  * score of key block j <= i is Qp_i . Kp_j.  The diagonal block i is always

@@ -59,6 +59,22 @@ def test_vs_32k_layer(orc, vs32k):
         check_attention(o2[0, rows], l2[0, rows], ref2[0], rl2[0], f"VS 32K head {h}, oracle indices")
 
 
+def test_vs_32k_layer_whole_tiles(orc, vs32k):
+    """The whole-slash-tile variant at full size on the GPU's own indices, sampled rows."""
+    w, x = vs32k
+    q, k, v = x["q"], x["k"], x["v"]
+    gv, gs = minf.minf_vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, SCALE)
+    out, lse = minf.minf_vs_attention_tiles(q, k, v, gv, gs, SCALE)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.n)
+    grp = w.hq // w.hkv
+    for h in (2, 29):
+        qh, kh, vh = head_inputs(x, h, grp)
+        ref, rl = orc.vs_tiles_attention(qh, kh, vh, SCALE, gv[h:h + 1].cpu().numpy(), gs[h:h + 1].cpu().numpy(),
+                                         128, rows=rows)
+        check_attention(out[h, rows], lse[h, rows], ref[0], rl[0], f"VS tiles 32K head {h}")
+
+
 def test_dense_32k_layer(orc, vs32k):
     w, x = vs32k
     out, lse = minf.minf_dense_attention(x["q"], x["k"], x["v"], SCALE)

@@ -333,3 +333,56 @@ def test_vs_attention_many_slash_groups(orc):
     out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
                                       scale=SCALE)
     check_attention(out[:, rows], lse[:, rows], ref, rl, "VS many groups")
+
+
+# ----------------------------------------------------------------------------- whole slash tiles
+@pytest.mark.parametrize("n,hq,hkv,nv,ns", [(1024, 4, 2, 40, 60), (1344, 2, 1, 100, 30), (4096, 1, 1, 256, 512),
+                                            (192, 2, 1, 8, 16), (64, 1, 1, 4, 8)])
+def test_vs_tiles_oracle_indices(orc, n, hq, hkv, nv, ns):
+    """Whole-slash-tile Vertical-Slash against the oracle's variant on the oracle's index sets."""
+    q, k, v = inputs(n, hq, hkv, seed=nv + 3)
+    vi, si = orc.vs_estimate(q, k, 64, nv, ns, SCALE)
+    ref, rl = orc.vs_tiles_attention(q, k, v, SCALE, vi, si, 128)
+    out, lse = minf.minf_vs_attention_tiles(*cuda(q, k, v), torch.from_numpy(vi).cuda(),
+                                            torch.from_numpy(si).cuda(), scale=SCALE)
+    check_attention(out, lse, ref, rl, f"VS tiles n={n}")
+
+
+def test_vs_tiles_unsorted_duplicates_and_far_offsets(orc):
+    """Unsorted rows with duplicates, -1 padding, offsets past n and a lone far offset."""
+    n, hq, hkv = 1088, 2, 1
+    q, k, v = inputs(n, hq, hkv, seed=78)
+    vi, si = _rand_vs_indices(np.random.default_rng(6), n, hq, 50, 70)
+    si[0, -1] = n + 100       # out of range: ignored
+    si[1, :] = -1
+    si[1, 0] = 300            # head 1: one far offset and the verticals
+    ref, rl = orc.vs_tiles_attention(q, k, v, SCALE, vi, si, 128)
+    out, lse = minf.minf_vs_attention_tiles(*cuda(q, k, v), torch.from_numpy(vi).cuda(),
+                                            torch.from_numpy(si).cuda(), scale=SCALE)
+    check_attention(out, lse, ref, rl, "VS tiles random sets")
+
+
+def test_vs_tiles_superset_of_exact():
+    """On the same indices the whole-tile key set contains the token-exact one: lse never drops."""
+    n = 2048
+    q, k, v = cuda(*inputs(n, 2, 1, seed=31))
+    gv, gs = minf.minf_vs_estimate(q, k, 64, 100, 300, scale=SCALE)
+    _, le = minf.minf_vs_attention(q, k, v, gv, gs, scale=SCALE)
+    _, lt = minf.minf_vs_attention_tiles(q, k, v, gv, gs, scale=SCALE)
+    assert torch.all(lt >= le - 1e-2)
+    assert torch.any(lt > le + 1e-2)
+
+
+def test_vs_tiles_many_slash_groups(orc):
+    """Over a thousand separate slash groups at 140K keys, sampled rows."""
+    n = 140096
+    q, k, v = inputs(n, 1, 1, seed=18)
+    offs = sorted(set([j * 130 for j in range(1078)] + [j * 130 + 60 for j in range(0, 1078, 7)]))
+    si = np.array([offs], np.int32)
+    rng = np.random.default_rng(5)
+    vi = np.sort(rng.choice(n, 64, replace=False)).astype(np.int32)[None, :]
+    rows = np.unique(np.concatenate([rng.integers(0, n, 200), np.arange(n - 64, n), [0, 127, 128, 140000]]))
+    ref, rl = orc.vs_tiles_attention(q, k, v, SCALE, vi, si, 128, rows=rows)
+    out, lse = minf.minf_vs_attention_tiles(*cuda(q, k, v), torch.from_numpy(vi).cuda(),
+                                            torch.from_numpy(si).cuda(), scale=SCALE)
+    check_attention(out[:, rows], lse[:, rows], ref, rl, "VS tiles many groups")
