@@ -45,6 +45,7 @@ _D = ctypes.c_double
 
 _SIGS = {
     "orc_vs_estimate": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _P, _I, _P, _P, _P, _P],
+    "orc_vs_estimate_topp": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _D, _D, _P, _I, _P, _P, _P, _P, _P, _P],
     "orc_block_estimate": [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P],
     "orc_dense_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _P, _I, _P, _P],
     "orc_ashape_attention": [_P, _P, _P, _I, _I, _I, _I, _D, _P, _I, _I, _I, _P, _I, _P, _P],
@@ -115,6 +116,28 @@ class Oracle:
         if return_scores:
             return v_idx, s_idx, vert, slash
         return v_idx, s_idx
+
+    def vs_estimate_topp(self, q, k, last_q: int, n_vertical: int, n_slash: int, p_vertical: float,
+                         p_slash: float, scale: float, head_ids=None, return_scores: bool = False):
+        """Top-p budgets: returns (v_idx, s_idx, v_cnt, s_cnt[, vert, slash])."""
+        q, k = self._f32(q), self._f32(k)
+        hq, n, d = q.shape
+        hkv = k.shape[0]
+        ids, nh = self._heads(hq, head_ids)
+        v_idx = np.empty((nh, n_vertical), np.int32)
+        s_idx = np.empty((nh, n_slash), np.int32)
+        v_cnt = np.empty(nh, np.int32)
+        s_cnt = np.empty(nh, np.int32)
+        vert = np.empty((nh, n), np.float64) if return_scores else None
+        slash = np.empty((nh, n), np.float64) if return_scores else None
+        rc = self.lib.orc_vs_estimate_topp(self._ptr(q), self._ptr(k), hq, hkv, n, d, last_q, n_vertical,
+                                           n_slash, p_vertical, p_slash, scale, self._ptr(ids), nh,
+                                           self._ptr(v_idx), self._ptr(s_idx), self._ptr(v_cnt),
+                                           self._ptr(s_cnt), self._ptr(vert), self._ptr(slash))
+        self._check(rc, "vs_estimate_topp")
+        if return_scores:
+            return v_idx, s_idx, v_cnt, s_cnt, vert, slash
+        return v_idx, s_idx, v_cnt, s_cnt
 
     # -- 2. Block-Sparse estimation ---------------------------------------------
     def block_estimate(self, q, k, block: int, topk: int, head_ids=None,

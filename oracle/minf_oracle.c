@@ -96,6 +96,36 @@ static void topk_ascending(scored_t *cand, int m, int kk, int *out, int cap) {
 
 /* ---- 1. Vertical-Slash estimation -------------------------------------------- */
 
+/* Column sums vert[k] and diagonal sums slash[o] of the row-softmax weights of
+ * the last L queries of one head (Q, K [n][d]); z is scratch of n doubles. */
+static void vs_scores(const float *Q, const float *K, int n, int d, int L, double scale, double *z,
+                      double *vert, double *slash) {
+    for (int i = n - L; i < n; ++i) {
+        /* logits of query i against keys 0..i (causal) */
+        double m = -INFINITY;
+#if ORC_MUTANT == 1 /* planted: no causal limit inside the last block */
+        const int kend = n - 1;
+#else
+        const int kend = i;
+#endif
+        for (int kk = 0; kk <= kend; ++kk) {
+            z[kk] = scale * dot(Q + (size_t)i * d, K + (size_t)kk * d, d);
+            if (z[kk] > m) m = z[kk];
+        }
+        double den = 0.0;
+        for (int kk = 0; kk <= kend; ++kk) den += exp(z[kk] - m);
+        for (int kk = 0; kk <= kend; ++kk) {
+            const double a = exp(z[kk] - m) / den; /* softmax weight A_ik */
+            vert[kk] += a;                          /* column sum */
+#if ORC_MUTANT == 2 /* planted: diagonal offset off by one */
+            slash[(i - kk + 1) % n] += a;
+#else
+            if (kk <= i) slash[i - kk] += a;        /* diagonal sum, o = i - k */
+#endif
+        }
+    }
+}
+
 int orc_vs_estimate(const float *q, const float *k, int hq, int hkv, int n, int d,
                     int last_q, int n_vertical, int n_slash, double scale,
                     const int *head_ids, int n_heads,
@@ -116,30 +146,7 @@ int orc_vs_estimate(const float *q, const float *k, int hq, int hkv, int n, int 
         if (!z || !vert || !slash || !cand) {
             failed = 1;
         } else {
-            for (int i = n - L; i < n; ++i) {
-                /* logits of query i against keys 0..i (causal) */
-                double m = -INFINITY;
-#if ORC_MUTANT == 1 /* planted: no causal limit inside the last block */
-                const int kend = n - 1;
-#else
-                const int kend = i;
-#endif
-                for (int kk = 0; kk <= kend; ++kk) {
-                    z[kk] = scale * dot(Q + (size_t)i * d, K + (size_t)kk * d, d);
-                    if (z[kk] > m) m = z[kk];
-                }
-                double den = 0.0;
-                for (int kk = 0; kk <= kend; ++kk) den += exp(z[kk] - m);
-                for (int kk = 0; kk <= kend; ++kk) {
-                    const double a = exp(z[kk] - m) / den; /* softmax weight A_ik */
-                    vert[kk] += a;                          /* column sum */
-#if ORC_MUTANT == 2 /* planted: diagonal offset off by one */
-                    slash[(i - kk + 1) % n] += a;
-#else
-                    if (kk <= i) slash[i - kk] += a;        /* diagonal sum, o = i - k */
-#endif
-                }
-            }
+            vs_scores(Q, K, n, d, L, scale, z, vert, slash);
 #if ORC_MUTANT != 3 /* planted (3): the main diagonal is not forced */
             slash[0] = INFINITY;
 #endif
@@ -147,6 +154,81 @@ int orc_vs_estimate(const float *q, const float *k, int hq, int hkv, int n, int 
             topk_ascending(cand, n, n_vertical, v_idx + (size_t)hp * n_vertical, n_vertical);
             for (int t = 0; t < n; ++t) { cand[t].s = slash[t]; cand[t].i = t; }
             topk_ascending(cand, n, n_slash, s_idx + (size_t)hp * n_slash, n_slash);
+            if (vert_out) memcpy(vert_out + (size_t)hp * n, vert, sizeof(double) * (size_t)n);
+            if (slash_out) memcpy(slash_out + (size_t)hp * n, slash, sizeof(double) * (size_t)n);
+        }
+        free(z); free(vert); free(slash); free(cand);
+    }
+    return failed ? ORC_ERR : ORC_OK;
+}
+
+/* Top-p selection: the shortest prefix of the (score desc, index asc) order of
+ * cand[first..m) whose score mass, added to `acc`, reaches `target`; at most
+ * cap - first entries.  cand must be sorted from `first` on.  Returns the
+ * number of entries taken. */
+static int topp_take(const scored_t *cand, int first, int m, double acc, double target, int cap) {
+    int c = first;
+    while (c < m && c < cap && acc < target) acc += cand[c++].s;
+    return c - first;
+}
+
+/* Vertical-Slash estimation with top-p budgets ([TALK], the part on the work
+ * that followed MInference: a top-p of the attention weights instead of a
+ * fixed top-k, with column-level estimation).  The scores are those of
+ * orc_vs_estimate.  Verticals: the fewest keys, best first (ties to the lower
+ * index), whose column sums reach p_vertical of the total column mass.
+ * Slashes: offset 0 first (forced, with its own mass), then the fewest further
+ * offsets, best first, until the diagonal mass reaches p_slash of the total.
+ * n_vertical and n_slash cap the counts and size the rows (-1 padded);
+ * v_cnt/s_cnt (nullable) get the counts; vert_out/slash_out (nullable) get the
+ * scores, slash_out[0] the true diagonal mass. */
+int orc_vs_estimate_topp(const float *q, const float *k, int hq, int hkv, int n, int d, int last_q,
+                         int n_vertical, int n_slash, double p_vertical, double p_slash, double scale,
+                         const int *head_ids, int n_heads, int *v_idx, int *s_idx, int *v_cnt,
+                         int *s_cnt, double *vert_out, double *slash_out) {
+    if (!q || !k || !v_idx || !s_idx || hq <= 0 || hkv <= 0 || hq % hkv || n <= 0 || d <= 0 ||
+        last_q <= 0 || n_vertical <= 0 || n_slash <= 0 || !(p_vertical > 0.0 && p_vertical <= 1.0) ||
+        !(p_slash > 0.0 && p_slash <= 1.0))
+        return ORC_ERR;
+    const int L = last_q < n ? last_q : n;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int hp = 0; hp < n_heads; ++hp) {
+        const int h = head_at(head_ids, hp), g = kv_of(h, hq, hkv);
+        const float *Q = q + (size_t)h * n * d, *K = k + (size_t)g * n * d;
+        double *z = (double *)malloc(sizeof(double) * (size_t)n);
+        double *vert = (double *)calloc((size_t)n, sizeof(double));
+        double *slash = (double *)calloc((size_t)n, sizeof(double));
+        scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)n);
+        if (!z || !vert || !slash || !cand) {
+            failed = 1;
+        } else {
+            vs_scores(Q, K, n, d, L, scale, z, vert, slash);
+            double tv = 0.0, ts = 0.0;
+            for (int t = 0; t < n; ++t) { tv += vert[t]; ts += slash[t]; }
+            int *vr = v_idx + (size_t)hp * n_vertical, *sr = s_idx + (size_t)hp * n_slash;
+            /* verticals */
+            for (int t = 0; t < n; ++t) { cand[t].s = vert[t]; cand[t].i = t; }
+            qsort(cand, (size_t)n, sizeof(scored_t), by_score_desc_index_asc);
+            const int cv = topp_take(cand, 0, n, 0.0, p_vertical * tv, n_vertical);
+            for (int j = 0; j < cv; ++j) vr[j] = cand[j].i;
+            qsort(vr, (size_t)cv, sizeof(int), int_asc);
+            for (int j = cv; j < n_vertical; ++j) vr[j] = -1;
+            /* slashes: offset 0, then the others best first */
+            for (int t = 1; t < n; ++t) { cand[t - 1].s = slash[t]; cand[t - 1].i = t; }
+            qsort(cand, (size_t)(n - 1), sizeof(scored_t), by_score_desc_index_asc);
+#if ORC_MUTANT == 9 /* planted: the forced diagonal's mass not counted */
+            const double acc0 = 0.0;
+#else
+            const double acc0 = slash[0];
+#endif
+            const int cs = topp_take(cand, 0, n - 1, acc0, p_slash * ts, n_slash - 1);
+            sr[0] = 0;
+            for (int j = 0; j < cs; ++j) sr[1 + j] = cand[j].i;
+            qsort(sr, (size_t)(cs + 1), sizeof(int), int_asc);
+            for (int j = cs + 1; j < n_slash; ++j) sr[j] = -1;
+            if (v_cnt) v_cnt[hp] = cv;
+            if (s_cnt) s_cnt[hp] = cs + 1;
             if (vert_out) memcpy(vert_out + (size_t)hp * n, vert, sizeof(double) * (size_t)n);
             if (slash_out) memcpy(slash_out + (size_t)hp * n, slash, sizeof(double) * (size_t)n);
         }

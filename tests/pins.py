@@ -301,6 +301,53 @@ def pin_vs_tiles_forms(orc):
     assert np.allclose(out, dense, rtol=1e-12, atol=1e-13), "every offset: dense"
 
 
+def pin_vs_topp_forms(orc):
+    """Top-p budgets ([TALK], work that followed MInference: a top-p of the attention
+    weights instead of a fixed top-k), against what the definition fixes:
+      * Q = 0 makes every row's softmax uniform, so vert[k] and slash[o] have closed
+        forms (sums of 1/(i+1)); the selected counts and sets follow from them, ties
+        to the lower index;
+      * the set is the top-k set of its own size (a prefix of the same order);
+      * it reaches p of the mass and is the shortest prefix that does;
+      * the caps bound the counts."""
+    n, L = 256, 64
+    rng = np.random.default_rng(3)
+    q = np.zeros((1, n, 128), np.float32)
+    k = rng.standard_normal((1, n, 128)).astype(np.float32)
+    rows = np.arange(n - L, n)
+    inv = 1.0 / (rows + 1.0)
+    vert = np.array([inv[rows >= kk].sum() for kk in range(n)])       # column kk: rows i >= kk
+    slash = np.array([inv[rows >= o].sum() for o in range(n)])       # offset o: rows i >= o
+    pv, ps = 0.5, 0.3
+    vi, si, vc, sc = orc.vs_estimate_topp(q, k, L, 200, 150, pv, ps, 0.1)
+    order = np.lexsort((np.arange(n), -vert))
+    cv = int(np.searchsorted(np.cumsum(vert[order]), pv * vert.sum(), side="left")) + 1
+    assert vc[0] == cv and np.array_equal(vi[0, :cv], np.sort(order[:cv])) and np.all(vi[0, cv:] == -1), \
+        "uniform rows: vertical count and set"
+    rest = np.arange(1, n)
+    order = rest[np.lexsort((rest, -slash[1:]))]
+    need = ps * slash.sum() - slash[0]
+    cs = int(np.searchsorted(np.cumsum(slash[order]), need, side="left")) + 1
+    assert sc[0] == cs + 1, "uniform rows: slash count (offset 0 forced, its mass counted)"
+    assert np.array_equal(si[0, :cs + 1], np.sort(np.concatenate([[0], order[:cs]]))), "uniform rows: slash set"
+    # planted inputs: prefix of the top-k order, minimal mass cover, caps
+    qq, kk_, _, _ = _inputs(512, hq=2, hkv=1, seed=41)
+    f32 = lambda a: a.astype(np.float32)
+    vi, si, vc, sc, vs, ss = orc.vs_estimate_topp(f32(qq), f32(kk_), 64, 512, 512, 0.9, 0.8, 1 / math.sqrt(128),
+                                                  return_scores=True)
+    for hp in range(2):
+        a, b = orc.vs_estimate(f32(qq), f32(kk_), 64, int(vc[hp]), int(sc[hp]), 1 / math.sqrt(128), head_ids=[hp])
+        assert np.array_equal(vi[hp, :vc[hp]], a[0]) and np.array_equal(si[hp, :sc[hp]], b[0]), "prefix of top-k"
+        sel = vs[hp, vi[hp, :vc[hp]]]
+        assert sel.sum() >= 0.9 * vs[hp].sum() and sel.sum() - sel.min() < 0.9 * vs[hp].sum(), "shortest vertical cover"
+        sel = ss[hp, si[hp, :sc[hp]]]
+        others = np.sort(ss[hp, si[hp, 1:sc[hp]]])
+        assert sel.sum() >= 0.8 * ss[hp].sum(), "slash cover"
+        assert len(others) == 0 or sel.sum() - others[0] < 0.8 * ss[hp].sum(), "shortest slash cover"
+    vi, si, vc, sc = orc.vs_estimate_topp(f32(qq), f32(kk_), 64, 5, 3, 0.99, 0.99, 1 / math.sqrt(128))
+    assert np.all(vc == 5) and np.all(sc == 3) and np.all(vi >= 0) and np.all(si[:, 0] == 0), "caps"
+
+
 def pin_full_budget_is_dense(orc):
     """Budgets that cover every key reduce each pattern to dense causal attention."""
     n = 320
@@ -370,6 +417,7 @@ ALL_PINS = [
     pin_full_budget_is_dense,
     pin_trishape_bruteforce,
     pin_vs_tiles_forms,
+    pin_vs_topp_forms,
     pin_attention_closed_forms,
     pin_planted_recovery,
 ]

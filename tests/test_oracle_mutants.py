@@ -4,7 +4,8 @@ The mutants are builds of the same C source with one plausible slip switched on
 (see ORC_MUTANT in minf_oracle.c): no causal limit in the estimate, an
 off-by-one diagonal, the main diagonal not forced, the Block-Sparse diagonal not
 forced, an A-shape window one key short, a key counted twice in Vertical-Slash,
-a Tri-shape tail one row short, a whole-slash-tile range one key too wide.
+a Tri-shape tail one row short, a whole-slash-tile range one key too wide,
+top-p slashes that ignore the forced diagonal's mass.
 """
 import pytest
 
@@ -20,6 +21,7 @@ MUTANTS = {
     6: "VS key counted twice",
     7: "Tri-shape dense tail one row short",
     8: "whole-slash-tile range one key too wide",
+    9: "top-p without the forced diagonal's mass",
 }
 
 
