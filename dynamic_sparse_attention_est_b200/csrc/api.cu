@@ -76,6 +76,8 @@ VsEstBufs carve_vs_est(Carver &c, int n, int n_heads, int n_pairs) {
     b.vert = c.take<float>((size_t)n_heads * n);
     b.slash = c.take<float>((size_t)n_heads * n);
     b.topk_scratch = c.take<char>(topk_scratch_bytes(n_heads, n));
+    b.diag0 = c.take<float>(n_heads);
+    b.counts = c.take<int>(2 * (size_t)n_heads);
     return b;
 }
 
@@ -268,7 +270,8 @@ int reset_counters(void *ws, cudaStream_t st) {
 // The bodies below assume checked arguments; `scratch` is the workspace past
 // the status header (or a sub-area of it in the mixed layer).
 int do_vs_estimate(const Common &c, const void *q, const void *k, int last_q, int nv, int ns, float scale,
-                   int32_t *v_idx, int32_t *s_idx, void *ws, char *scratch, cudaStream_t st) {
+                   int32_t *v_idx, int32_t *s_idx, void *ws, char *scratch, cudaStream_t st, float p_v = 0.f,
+                   float p_s = 0.f, int32_t *v_cnt = nullptr, int32_t *s_cnt = nullptr) {
     // count the pairs the estimate kernel will form
     const int group = c.hq / c.hkv;
     int n_pairs = 0;
@@ -293,6 +296,11 @@ int do_vs_estimate(const Common &c, const void *q, const void *k, int last_q, in
     a.n_slash = ns;
     a.v_idx = v_idx;
     a.s_idx = s_idx;
+    a.topp = p_v > 0.f;
+    a.p_vertical = p_v;
+    a.p_slash = p_s;
+    a.v_cnt = v_cnt;
+    a.s_cnt = s_cnt;
     a.hdr = ws;
     a.wait_limit_ns = g_wait_limit_ns.load();
     cudaError_t e = run_vs_estimate(a, b, st);
@@ -482,6 +490,28 @@ int minf_vs_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, in
     if ((rc = select_device(q))) return rc;
     return do_vs_estimate(c, q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws,
                           static_cast<char *>(ws) + MINF_STATUS_BYTES, (cudaStream_t)stream);
+}
+
+int minf_vs_estimate_topp(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d, int last_q,
+                          int n_vertical, int n_slash, float p_vertical, float p_slash, float scale,
+                          const int32_t *head_ids, int n_heads, int32_t *v_idx, int32_t *s_idx, int32_t *v_cnt,
+                          int32_t *s_cnt, void *ws, size_t ws_bytes, minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if ((rc = check_scale(scale))) return rc;
+    if (!v_idx || !s_idx) return fail(MINF_ERR_INVALID, "null v_idx or s_idx");
+    if (n_vertical < 1 || n_slash < 1) return fail(MINF_ERR_INVALID, "caps must be >= 1");
+    if (!(p_vertical > 0.f && p_vertical <= 1.f) || !(p_slash > 0.f && p_slash <= 1.f))
+        return fail(MINF_ERR_INVALID, "p must be in (0, 1]");
+    if (last_q < 1) return fail(MINF_ERR_INVALID, "last_q must be >= 1");
+    if (last_q > 64) return fail(MINF_ERR_UNSUPPORTED, "last_q %d above 64", last_q);
+    if (n > (1 << 20)) return fail(MINF_ERR_UNSUPPORTED, "top-p rows above 2^20 keys");
+    if ((rc = check_ws(ws, ws_bytes, bytes_vs_est(hkv, n, c.n_heads)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    return do_vs_estimate(c, q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws,
+                          static_cast<char *>(ws) + MINF_STATUS_BYTES, (cudaStream_t)stream, p_vertical, p_slash,
+                          v_cnt, s_cnt);
 }
 
 static int vs_attention_entry(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv,

@@ -40,6 +40,8 @@ struct VsEstBufs {
     float *vert;    // [n_heads][n]
     float *slash;   // [n_heads][n]
     void *topk_scratch;  // topk_scratch_bytes(n_heads, n)
+    float *diag0;   // [n_heads] mass of offset 0 (its slash entry is forced to +inf)
+    int *counts;    // [2][n_heads] top-p counts when the caller keeps none
     int n_chunks, chunk_tiles, n_ktiles;
 };
 
@@ -50,6 +52,9 @@ struct VsEstArgs {
     const int *head_ids;   // host, n_heads entries
     int n_vertical, n_slash;
     int *v_idx, *s_idx;
+    bool topp;             // budgets by mass: p_vertical / p_slash, n_vertical / n_slash as caps
+    float p_vertical, p_slash;
+    int *v_cnt, *s_cnt;    // device, nullable: the top-p counts
     void *hdr;             // WsHeader*
     unsigned long long wait_limit_ns;
 };
@@ -83,8 +88,15 @@ cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaS
 // non-negative floats each; writes min(k, len) indices ascending, -1 padded to k.
 // Rows longer than the one-block limit need topk_scratch_bytes(n_rows, len)
 // bytes of device scratch (256-byte aligned); shorter rows need none.
+// With k_row (device, n_rows entries) row r keeps min(k_row[r], k) keys.
 size_t topk_scratch_bytes(int n_rows, int len);
 cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
-                          cudaStream_t st);
+                          cudaStream_t st, const int *k_row = nullptr);
+
+// Top-p counts (device, n_rows entries, each at most cap): the fewest keys of a
+// row, best first, whose scores reach p of the row's mass; with skip0 key 0 is
+// left out and extra0[r] counts first (the count then includes that entry).
+cudaError_t run_topp_counts(const float *scores, int n_rows, int len, bool skip0, const float *extra0, float p,
+                            int cap, int *count, cudaStream_t st);
 
 }  // namespace minf

@@ -27,7 +27,7 @@ constexpr int kChunk = 8192;         // keys per block in the multi-block path
 constexpr int kChunkThreads = 256;
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_smem_kernel(const float *scores, int len, int k,
-                                                                      int *out) {
+                                                                      const int *k_row, int *out) {
     extern __shared__ float row[];
     __shared__ TopkShared sh;
     const float *x = scores + (size_t)blockIdx.x * len;
@@ -40,21 +40,23 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_smem_kernel(const floa
     }
     __syncthreads();
     int *o = out + (size_t)blockIdx.x * k;
-    block_topk_ascending<kTopkThreads, false>(row, len, k, o, 0, sh);
-    for (int j = min(k, len) + (int)threadIdx.x; j < k; j += kTopkThreads) o[j] = -1;
+    const int kr = k_row ? max(0, min(k_row[blockIdx.x], k)) : k;
+    block_topk_ascending<kTopkThreads, false>(row, len, kr, o, 0, sh);
+    for (int j = min(kr, len) + (int)threadIdx.x; j < k; j += kTopkThreads) o[j] = -1;
 }
 
 // ---- multi-block path --------------------------------------------------------
 struct RowState {
     uint32_t prefix, mask;
     int remaining;  // keys equal to the threshold still to take
-    int pad;
+    int k;          // this row's count, at most the row stride
 };
 
-__global__ void topk_init_kernel(RowState *st, uint32_t *hist, int rows, int len, int k) {
+__global__ void topk_init_kernel(RowState *st, uint32_t *hist, int rows, int len, int k, const int *k_row) {
     const int r = blockIdx.x;
     for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[(size_t)r * 256 + b] = 0u;
-    if (threadIdx.x == 0) st[r] = RowState{0u, 0u, min(k, len), 0};
+    const int kr = k_row ? max(0, min(k_row[r], k)) : k;
+    if (threadIdx.x == 0) st[r] = RowState{0u, 0u, min(kr, len), kr};
 }
 
 __global__ void __launch_bounds__(kChunkThreads) topk_hist_kernel(const float *scores, int len,
@@ -117,7 +119,8 @@ __global__ void __launch_bounds__(kChunkThreads) topk_count_kernel(const float *
                                                                    int2 *cnt, int n_chunks) {
     __shared__ int red[2][kChunkThreads / 32];
     const int r = blockIdx.y;
-    const uint32_t t = st[r].prefix;
+    // a row with nothing to take: every key counts as below the threshold
+    const uint32_t t = st[r].k > 0 ? st[r].prefix : 0xffffffffu;
     const float *x = scores + (size_t)r * len;
     const int c0 = blockIdx.x * kChunk, c1 = min(len, c0 + kChunk);
     int gt = 0, eq = 0;
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kChunkThreads) topk_write_kernel(const float *
                                                                    int n_chunks, int *out) {
     __shared__ TopkShared sh;
     const int r = blockIdx.y;
-    const uint32_t t = st[r].prefix;
+    const uint32_t t = st[r].k > 0 ? st[r].prefix : 0xffffffffu;
     const int need = st[r].remaining;
     const int2 base = off[(size_t)r * n_chunks + blockIdx.x];
     const float *x = scores + (size_t)r * len;
@@ -203,10 +206,160 @@ __global__ void __launch_bounds__(kChunkThreads) topk_write_kernel(const float *
         eq_seen += eq_tot;
     }
     if (blockIdx.x == 0)
-        for (int j = min(k, len) + (int)threadIdx.x; j < k; j += kChunkThreads) o[j] = -1;
+        for (int j = min(st[r].k, len) + (int)threadIdx.x; j < k; j += kChunkThreads) o[j] = -1;
+}
+
+// ---- top-p counts -------------------------------------------------------------
+// For each row: the fewest keys, best first (ties to the lower index), whose
+// scores sum to at least p of the row's mass.  With skip0, key 0 is left out
+// (it holds a forced entry) and extra0[row], that entry's own score, is counted
+// first.  Masses are summed exactly in 2^-32 fixed point (a score is at most
+// 64, so a row of 2^20 keys stays below 2^58): the count does not depend on
+// the order of the additions.  The threshold is found like the top-k one, on
+// histograms of mass instead of counts, one 1024-thread CTA per row.
+constexpr int kToppThreads = 1024;
+
+__device__ __forceinline__ unsigned long long fixed_mass(float x) {
+    return __float2ull_rz(x * 4294967296.0f);
+}
+
+__device__ __forceinline__ unsigned long long shfl_up_u64(unsigned long long v, int d) {
+    const uint32_t lo = __shfl_up_sync(0xffffffffu, (uint32_t)v, d);
+    const uint32_t hi = __shfl_up_sync(0xffffffffu, (uint32_t)(v >> 32), d);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+__global__ void __launch_bounds__(kToppThreads) topp_count_kernel(const float *scores, int len, int skip0,
+                                                                 const float *extra0, float p, int cap,
+                                                                 int *count) {
+    __shared__ unsigned long long hmass[256];
+    __shared__ uint32_t hcnt[256];
+    __shared__ unsigned long long red[kToppThreads / 32];
+    __shared__ unsigned long long s_rem;
+    __shared__ uint32_t s_prefix, s_mask;
+    __shared__ int s_above, s_done, s_eq;
+    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float *x = scores + (size_t)r * len;
+    const int first = skip0 ? 1 : 0;
+    // total mass of the candidates
+    unsigned long long part = 0;
+    for (int i = first + tid; i < len; i += kToppThreads) part += fixed_mass(__ldg(x + i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) red[wid] = part;
+    __syncthreads();
+    if (tid == 0) {
+        unsigned long long total = 0;
+        for (int w = 0; w < kToppThreads / 32; ++w) total += red[w];
+        const unsigned long long m0 = skip0 ? fixed_mass(extra0[r]) : 0ull;
+        unsigned long long target = (unsigned long long)ceil((double)p * (double)(total + m0));
+        target = min(target, total + m0);
+        s_rem = target > m0 ? target - m0 : 0ull;
+        s_prefix = 0u;
+        s_mask = 0u;
+        s_above = 0;
+        s_done = s_rem == 0ull;
+        s_eq = 0;
+    }
+    __syncthreads();
+    for (int pass = 0; pass < 4 && !s_done; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int b = tid; b < 256; b += kToppThreads) {
+            hmass[b] = 0ull;
+            hcnt[b] = 0u;
+        }
+        __syncthreads();
+        const uint32_t prefix = s_prefix, pmask = s_mask;
+        for (int i0 = first; i0 < len; i0 += kToppThreads) {
+            const int i = i0 + tid;
+            uint32_t u = 0u;
+            bool valid = false;
+            if (i < len) {
+                u = __float_as_uint(__ldg(x + i));
+                valid = (u & pmask) == prefix;
+            }
+            const uint32_t bin = (u >> shift) & 255u;
+            const unsigned long long m = valid ? fixed_mass(__uint_as_float(u)) : 0ull;
+            // one atomic per distinct bin per warp: exact sums of <= 2^16 / 2^16 / 2^6 parts
+            unsigned todo = __ballot_sync(0xffffffffu, valid);
+            while (todo) {
+                const int leader = __ffs(todo) - 1;
+                const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+                const bool mine = valid && bin == lb;
+                const unsigned grp = __ballot_sync(0xffffffffu, mine);
+                const uint32_t a = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m & 0xffffu) : 0u);
+                const uint32_t b = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)((m >> 16) & 0xffffu) : 0u);
+                const uint32_t c = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m >> 32) : 0u);
+                if (lane == leader) {
+                    atomicAdd(&hcnt[lb], (uint32_t)__popc(grp));
+                    atomicAdd(&hmass[lb], ((unsigned long long)c << 32) + ((unsigned long long)b << 16) + a);
+                }
+                todo &= ~grp;
+            }
+        }
+        __syncthreads();
+        if (wid == 0) {
+            // lane L owns bins 255-8L .. 248-8L; scan from the top for the bin where the mass is reached
+            unsigned long long ms[8], sum = 0;
+            uint32_t cs[8], csum = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ms[e] = hmass[255 - 8 * lane - e];
+                cs[e] = hcnt[255 - 8 * lane - e];
+                sum += ms[e];
+                csum += cs[e];
+            }
+            unsigned long long incl = sum;
+            uint32_t cincl = csum;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const unsigned long long y = shfl_up_u64(incl, d);
+                const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, d);
+                if (lane >= d) {
+                    incl += y;
+                    cincl += cy;
+                }
+            }
+            const unsigned long long rem = s_rem;
+            unsigned long long cum = incl - sum;
+            uint32_t ccum = cincl - csum;
+            if (cum < rem && incl >= rem) {
+                int e = 0;
+                for (; e < 7; ++e) {
+                    if (cum + ms[e] >= rem) break;
+                    cum += ms[e];
+                    ccum += cs[e];
+                }
+                s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
+                s_mask = pmask | (255u << shift);
+                s_rem = rem - cum;
+                s_above += (int)ccum;
+                s_eq = (int)cs[e];
+            }
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        int c = 0;
+        if (!s_done) {
+            // keys above the threshold, then as many of its ties (each of the same mass) as the rest needs
+            const unsigned long long mt = fixed_mass(__uint_as_float(s_prefix));
+            long long need = mt ? (long long)((s_rem + mt - 1) / mt) : (long long)s_eq;
+            need = min(need, (long long)s_eq);
+            c = s_above + (int)need;
+        }
+        count[r] = min(c + (skip0 ? 1 : 0), cap);
+    }
 }
 
 }  // namespace
+
+cudaError_t run_topp_counts(const float *scores, int n_rows, int len, bool skip0, const float *extra0, float p,
+                            int cap, int *count, cudaStream_t st) {
+    if (n_rows <= 0) return cudaSuccess;
+    topp_count_kernel<<<n_rows, kToppThreads, 0, st>>>(scores, len, skip0 ? 1 : 0, extra0, p, cap, count);
+    return cudaGetLastError();
+}
 
 size_t topk_scratch_bytes(int n_rows, int len) {
     if (len <= kSmemRow) return 0;
@@ -215,13 +368,13 @@ size_t topk_scratch_bytes(int n_rows, int len) {
 }
 
 cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int *k_row) {
     if (n_rows <= 0 || k <= 0) return cudaSuccess;
     if (len <= kSmemRow) {
         const int smem = len * (int)sizeof(float);
         cudaError_t e = cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        topk_rows_smem_kernel<<<n_rows, kTopkThreads, smem, st>>>(scores, len, k, out);
+        topk_rows_smem_kernel<<<n_rows, kTopkThreads, smem, st>>>(scores, len, k, k_row, out);
         return cudaGetLastError();
     }
     if (!scratch) return cudaErrorInvalidValue;
@@ -236,7 +389,7 @@ cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *
     int2 *cnt = reinterpret_cast<int2 *>(p + off);
     off = align(off + (size_t)n_rows * n_chunks * sizeof(int2));
     int2 *offs = reinterpret_cast<int2 *>(p + off);
-    topk_init_kernel<<<n_rows, 256, 0, st>>>(state, hist, n_rows, len, k);
+    topk_init_kernel<<<n_rows, 256, 0, st>>>(state, hist, n_rows, len, k, k_row);
     const dim3 grid(n_chunks, n_rows);
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;

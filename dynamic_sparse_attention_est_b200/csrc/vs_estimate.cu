@@ -255,7 +255,7 @@ __global__ void lse_combine_kernel(const float2 *part, int n_pairs, int n_chunks
 
 // slash[hp][o] = sum of the (at most two) key tiles' diagonal partials that
 // cover offset o, in increasing tile order; offset 0 is forced to +inf.
-__global__ void slash_combine_kernel(const float *diag, int n, int n_ktiles, float *slash) {
+__global__ void slash_combine_kernel(const float *diag, int n, int n_ktiles, float *slash, float *diag0) {
     const int hp = blockIdx.y;
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
     if (o >= n) return;
@@ -265,7 +265,8 @@ __global__ void slash_combine_kernel(const float *diag, int n, int n_ktiles, flo
         const int rel = o - (n - kDiagW - kt * 128);
         if (rel >= 0 && rel < kDiagW) s += diag[((size_t)hp * n_ktiles + kt) * kDiagW + rel];
     }
-    slash[(size_t)hp * n + o] = o == 0 ? INFINITY : s;
+    slash[(size_t)hp * n + o] = o == 0 ? INFINITY : s;  // offset 0 is forced
+    if (o == 0) diag0[hp] = s;                           // its mass, for top-p budgets
 }
 
 }  // namespace
@@ -318,12 +319,23 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
     lse_combine_kernel<<<(np * 128 + 255) / 256, 256, 0, st>>>(b.part, np, b.n_chunks, b.lse2);
     vs_est_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(P);
     dim3 sg((a.n + 255) / 256, a.n_heads);
-    slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash);
+    slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash, b.diag0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, b.topk_scratch, st);
+    const int *kv = nullptr, *ks = nullptr;
+    if (a.topp) {
+        // top-p: per-row counts by mass, then the same ordered selection with those counts
+        int *cv = a.v_cnt ? a.v_cnt : b.counts, *cs = a.s_cnt ? a.s_cnt : b.counts + a.n_heads;
+        e = run_topp_counts(b.vert, a.n_heads, a.n, false, nullptr, a.p_vertical, a.n_vertical, cv, st);
+        if (e == cudaSuccess)
+            e = run_topp_counts(b.slash, a.n_heads, a.n, true, b.diag0, a.p_slash, a.n_slash, cs, st);
+        if (e != cudaSuccess) return e;
+        kv = cv;
+        ks = cs;
+    }
+    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, b.topk_scratch, st, kv);
     if (e != cudaSuccess) return e;
-    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, b.topk_scratch, st);
+    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, b.topk_scratch, st, ks);
 }
 
 }  // namespace minf

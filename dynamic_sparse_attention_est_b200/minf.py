@@ -44,6 +44,8 @@ _SIGS = {
     "minf_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "minf_vs_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_vs_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "minf_vs_estimate_topp": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _F, _P, _I, _P, _P, _P, _P, _P, _SZ,
+                                   _P]),
     "minf_vs_attention_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
@@ -155,6 +157,26 @@ def minf_vs_estimate(q, k, last_q: int = 64, n_vertical: int = 1000, n_slash: in
                                   ids, nh, _ptr(v_idx), _ptr(s_idx), _ptr(ws), ws.numel(), _stream(q.device)),
            "minf_vs_estimate")
     return v_idx, s_idx
+
+
+def minf_vs_estimate_topp(q, k, last_q: int = 64, n_vertical: int = 1000, n_slash: int = 6096,
+                          p_vertical: float = 0.9, p_slash: float = 0.9, scale: Optional[float] = None,
+                          head_ids=None, ws=None):
+    """Top-p budgets (the budgets are caps); returns (v_idx, s_idx, v_cnt, s_cnt)."""
+    hq, hkv, n, d = _qkv(q, k)
+    ids, nh = _heads(hq, head_ids)
+    need = workspace_bytes(OP_VS_ESTIMATE, hq, hkv, n, nh)
+    ws = _ws_for(ws, need, q.device)
+    v_idx = torch.empty(nh, n_vertical, dtype=torch.int32, device=q.device)
+    s_idx = torch.empty(nh, n_slash, dtype=torch.int32, device=q.device)
+    v_cnt = torch.empty(nh, dtype=torch.int32, device=q.device)
+    s_cnt = torch.empty(nh, dtype=torch.int32, device=q.device)
+    _check(lib().minf_vs_estimate_topp(_ptr(q), _ptr(k), hq, hkv, n, d, last_q, n_vertical, n_slash,
+                                       float(p_vertical), float(p_slash), _scale(scale), ids, nh, _ptr(v_idx),
+                                       _ptr(s_idx), _ptr(v_cnt), _ptr(s_cnt), _ptr(ws), ws.numel(),
+                                       _stream(q.device)),
+           "minf_vs_estimate_topp")
+    return v_idx, s_idx, v_cnt, s_cnt
 
 
 def minf_vs_estimate_noalloc(q, k, last_q: int = 64, n_vertical: int = 1000, n_slash: int = 6096,

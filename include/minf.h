@@ -109,6 +109,25 @@ int minf_vs_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, in
                      void *ws, size_t ws_bytes, minf_stream_t stream);
 
 /*
+ * Vertical-Slash index estimation with top-p budgets ([TALK], the part on the
+ * work that followed MInference: a top-p of the attention weights instead of a
+ * fixed top-k).  The scores are those of minf_vs_estimate.  Verticals: the
+ * fewest keys, best first (ties to the lower index), whose column sums reach
+ * p_vertical of the total column mass.  Slashes: offset 0 (forced, its own
+ * diagonal mass counted), then the fewest further offsets, best first, until
+ * the diagonal mass reaches p_slash of the total.  n_vertical and n_slash are
+ * caps: they size the rows (ASCENDING, -1 padded, as minf_vs_estimate) and
+ * bound the counts.  v_cnt, s_cnt (device int32 [n_heads], nullable) receive
+ * the counts.  0 < p <= 1; n <= 2^20 (masses are summed exactly in 2^-32
+ * fixed point).  Workspace: MINF_OP_VS_ESTIMATE.
+ */
+int minf_vs_estimate_topp(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                          int last_q, int n_vertical, int n_slash, float p_vertical, float p_slash,
+                          float scale, const int32_t *head_ids, int n_heads, int32_t *v_idx,
+                          int32_t *s_idx, int32_t *v_cnt, int32_t *s_cnt, void *ws,
+                          size_t ws_bytes, minf_stream_t stream);
+
+/*
  * Vertical-Slash sparse attention.  Query i of head position p attends to
  * key k iff k <= i and (k is in v_idx[p] or i - k is in s_idx[p]); each such
  * key once.  Entries < 0 in the index rows are ignored; rows need not be

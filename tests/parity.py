@@ -26,6 +26,9 @@ def to_np(t):
     return np.asarray(t, dtype=np.float64)
 
 
+MASS_TOL = 2e-5  # fp32 column / diagonal sums against the fp64 ones, as a share of the row mass
+
+
 def check_attention(gpu_out, gpu_lse, ref_out, ref_lse, what=""):
     g = to_np(gpu_out)
     r = np.asarray(ref_out, np.float64)
@@ -66,3 +69,33 @@ def check_topk_band(gpu_idx, scores, k, what=""):
     assert not miss, f"{what}: missing clear winners {miss[:10]}"
     assert not extra, f"{what}: took clear losers {extra[:10]}"
     return len(got) - len(set(must.tolist()) & gs)  # picks decided inside the band
+
+
+def check_topp(gpu_idx, gpu_cnt, scores, p, cap, forced0=False, what=""):
+    """Top-p parity.  gpu_idx: 1-D indices (-1 padded); gpu_cnt: the GPU's count;
+    scores: the oracle's fp64 scores of every candidate (for slashes the true
+    mass of offset 0, which is forced when forced0).
+
+    The GPU set must be the top-c set of the oracle's order for its own count c
+    (tie band), and c must be the shortest cover of p of the mass under the
+    oracle's scores, within the fp32 rounding of the scores (MASS_TOL of the total).
+    """
+    scores = np.asarray(scores, np.float64)
+    idx = np.asarray(gpu_idx).ravel()
+    c = int(gpu_cnt)
+    assert 1 <= c <= cap, f"{what}: count {c} outside [1, {cap}]"
+    got = idx[:c]
+    assert np.all(got >= 0) and np.all(idx[c:] == -1), f"{what}: count and padding disagree"
+    ranked = scores.copy()
+    if forced0:
+        ranked[0] = np.inf
+        assert 0 in set(got.tolist()), f"{what}: forced offset 0 missing"
+    check_topk_band(idx, ranked, c, what)
+    total = scores.sum()
+    mass = scores[got].sum()
+    tol = MASS_TOL * total
+    if c < cap:
+        assert mass >= p * total - tol, f"{what}: mass {mass:.6g} below p*total {p * total:.6g}"
+    rest = np.sort(scores[got[got != 0]] if forced0 else scores[got])
+    if len(rest):
+        assert mass - rest[0] < p * total + tol, f"{what}: not the shortest cover"

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from dynamic_sparse_attention_est_b200 import minf, synth
-from parity import check_attention, check_topk_band, to_np
+from parity import check_attention, check_topk_band, check_topp, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -386,3 +386,45 @@ def test_vs_tiles_many_slash_groups(orc):
     out, lse = minf.minf_vs_attention_tiles(*cuda(q, k, v), torch.from_numpy(vi).cuda(),
                                             torch.from_numpy(si).cuda(), scale=SCALE)
     check_attention(out[:, rows], lse[:, rows], ref, rl, "VS tiles many groups")
+
+
+# ----------------------------------------------------------------------------- top-p budgets
+@pytest.mark.parametrize("n,hq,hkv,pv,ps,cv,cs", [(1024, 4, 2, 0.9, 0.9, 1024, 1024), (4096, 1, 1, 0.5, 0.95, 4096, 4096),
+                                                  (2048, 2, 1, 0.99, 0.99, 40, 30),
+                                                  (65600, 1, 1, 0.8, 0.7, 65600, 65600)])
+def test_vs_estimate_topp(orc, n, hq, hkv, pv, ps, cv, cs):
+    q, k, _ = inputs(n, hq, hkv, seed=n + 7)
+    vi, si, vc, sc, vert, slash = orc.vs_estimate_topp(q, k, 64, cv, cs, pv, ps, SCALE, return_scores=True)
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(*cuda(q, k), 64, cv, cs, pv, ps, scale=SCALE)
+    gv, gs, gvc, gsc = gv.cpu().numpy(), gs.cpu().numpy(), gvc.cpu().numpy(), gsc.cpu().numpy()
+    for hp in range(hq):
+        check_topp(gv[hp], gvc[hp], vert[hp], pv, cv, False, f"top-p vertical h{hp}")
+        check_topp(gs[hp], gsc[hp], slash[hp], ps, cs, True, f"top-p slash h{hp}")
+        assert abs(int(gvc[hp]) - int(vc[hp])) <= max(2, vc[hp] // 200), "vertical count near the oracle's"
+        assert abs(int(gsc[hp]) - int(sc[hp])) <= max(2, sc[hp] // 200), "slash count near the oracle's"
+
+
+def test_vs_topp_exact_ties_uniform_rows(orc):
+    """Q = 0: every key column the last rows all see ties exactly (each column is summed
+    over the same rows in the same order), so the vertical top-p set is the oracle's:
+    the lowest indices among the ties, and the same count.  The diagonal sums are
+    assembled from per-tile partials in an order that depends on the offset, so the
+    slashes are checked within the band."""
+    n = 4096
+    q, k, _ = inputs(n, 1, 1, seed=12)
+    q = torch.zeros_like(q)
+    vi, si, vc, sc, vert, slash = orc.vs_estimate_topp(q, k, 64, 3000, 3000, 0.5, 0.3, SCALE, return_scores=True)
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(*cuda(q, k), 64, 3000, 3000, 0.5, 0.3, scale=SCALE)
+    assert int(gvc[0]) == int(vc[0]) and np.array_equal(gv[0].cpu().numpy(), vi[0])
+    check_topp(gs[0].cpu().numpy(), gsc[0].item(), slash[0], 0.3, 3000, True, "uniform rows, slashes")
+
+
+def test_vs_topp_then_attention(orc):
+    """Top-p indices feed the attention unchanged (-1 padding ignored)."""
+    n = 2048
+    q, k, v = inputs(n, 2, 1, seed=19)
+    vi, si, _, _ = orc.vs_estimate_topp(q, k, 64, 512, 512, 0.9, 0.9, SCALE)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out, lse, ref, rl, "VS attention on top-p indices")
