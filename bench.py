@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--workload", default="vs-gqa-32k")
     ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--topp", type=float, default=None,
+                    help="Vertical-Slash top-p budgets (p for verticals and slashes; the budgets become caps)")
     ap.add_argument("--vs-mode", default="exact", choices=["exact", "tiles"],
                     help="Vertical-Slash key set: token-exact, or every computed slash range attended whole")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-kernel comparison")
@@ -142,7 +144,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workload
-def make_step(w, x, torch, minf, synth, seed, vs_mode="exact"):
+def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None):
     """Returns (step(ws) -> out, attention-only call for timing, label of the attention call)."""
     q, k, v = x["q"], x["k"], x["v"]
     hq, hkv, n = w.hq, w.hkv, w.n
@@ -156,7 +158,12 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact"):
         state = {}
 
         def estimate():
-            state["idx"] = minf.minf_vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, scale, ws=ws_est)
+            if topp is None:
+                state["idx"] = minf.minf_vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, scale, ws=ws_est)
+            else:
+                vi, si, _, _ = minf.minf_vs_estimate_topp(q, k, w.last_q, w.n_vertical, w.n_slash, topp, topp,
+                                                          scale, ws=ws_est)
+                state["idx"] = (vi, si)
 
         vs_attention = minf.minf_vs_attention_tiles if vs_mode == "tiles" else minf.minf_vs_attention
 
@@ -164,7 +171,9 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact"):
             vi, si = state["idx"]
             vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
 
-        return estimate, attend, ws, out, 6, 4
+        # launches: 4 estimate kernels, two top-k rows (1 kernel up to 48K keys, else 12), top-p counts
+        topk_k = 1 if n <= 48 * 1024 else 12
+        return estimate, attend, ws, out, 4 + 2 * topk_k + (2 if topp is not None else 0), 4
     if w.pattern == "block":
         ws_est = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ESTIMATE, hq, hkv, n, hq, w.topk), dev)
         ws = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ATTENTION, hq, hkv, n, hq, w.topk), dev)
@@ -348,7 +357,7 @@ def main():
     x = synth.generate(w, seed=seed, device=dev)
     torch.cuda.synchronize()
     log("inputs ready")
-    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed, args.vs_mode)
+    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed, args.vs_mode, args.topp)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -403,7 +412,7 @@ def main():
         host_in = {key: x[key].cpu().pin_memory() for key in ("q", "k", "v")}
         x2 = {key: torch.empty_like(x[key]) for key in ("q", "k", "v")}
         sets = [(x, estimate, attend, out)]
-        e2, a2, _, o2, _, _ = make_step(w, x2, torch, minf, synth, seed, args.vs_mode)
+        e2, a2, _, o2, _, _ = make_step(w, x2, torch, minf, synth, seed, args.vs_mode, args.topp)
         sets.append((x2, e2, a2, o2))
         host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -497,6 +506,8 @@ def main():
                        "last_q": w.last_q, "n_vertical": w.n_vertical, "n_slash": w.n_slash, "topk": w.topk,
                        "n_sink": w.n_sink, "window": w.window,
                        **({"vs_mode": args.vs_mode} if w.pattern == "vs" else {}),
+                       **({"budgets": f"top-p {args.topp} (n_vertical, n_slash as caps)"}
+                          if w.pattern == "vs" and args.topp is not None else {}),
                        "l2": "inputs larger than L2 (no flush)",
                        "parallelism": f"one layer per rank x{world}"},
             "roofline": roofline,

@@ -78,6 +78,7 @@ VsEstBufs carve_vs_est(Carver &c, int n, int n_heads, int n_pairs) {
     b.topk_scratch = c.take<char>(topk_scratch_bytes(n_heads, n));
     b.diag0 = c.take<float>(n_heads);
     b.counts = c.take<int>(2 * (size_t)n_heads);
+    b.topp_scratch = c.take<char>(topp_scratch_bytes(n_heads));
     return b;
 }
 

@@ -42,6 +42,7 @@ struct VsEstBufs {
     void *topk_scratch;  // topk_scratch_bytes(n_heads, n)
     float *diag0;   // [n_heads] mass of offset 0 (its slash entry is forced to +inf)
     int *counts;    // [2][n_heads] top-p counts when the caller keeps none
+    void *topp_scratch;  // topp_scratch_bytes(n_heads)
     int n_chunks, chunk_tiles, n_ktiles;
 };
 
@@ -96,7 +97,9 @@ cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *
 // Top-p counts (device, n_rows entries, each at most cap): the fewest keys of a
 // row, best first, whose scores reach p of the row's mass; with skip0 key 0 is
 // left out and extra0[r] counts first (the count then includes that entry).
+// scratch: topp_scratch_bytes(n_rows) bytes of device memory, 256-byte aligned.
+size_t topp_scratch_bytes(int n_rows);
 cudaError_t run_topp_counts(const float *scores, int n_rows, int len, bool skip0, const float *extra0, float p,
-                            int cap, int *count, cudaStream_t st);
+                            int cap, int *count, void *scratch, cudaStream_t st);
 
 }  // namespace minf

@@ -216,8 +216,17 @@ __global__ void __launch_bounds__(kChunkThreads) topk_write_kernel(const float *
 // first.  Masses are summed exactly in 2^-32 fixed point (a score is at most
 // 64, so a row of 2^20 keys stays below 2^58): the count does not depend on
 // the order of the additions.  The threshold is found like the top-k one, on
-// histograms of mass instead of counts, one 1024-thread CTA per row.
-constexpr int kToppThreads = 1024;
+// histograms of mass instead of counts, over 8K-key chunks of the row.
+constexpr int kToppChunk = 8192;
+
+struct ToppState {
+    uint32_t prefix, mask;
+    unsigned long long rem;  // mass still needed from keys at or below the current prefix
+    int above;               // keys already known to be above the threshold
+    int eq;                  // keys in the chosen bin of the last pass
+    int done;                // nothing (more) needed
+    int pad;
+};
 
 __device__ __forceinline__ unsigned long long fixed_mass(float x) {
     return __float2ull_rz(x * 4294967296.0f);
@@ -229,135 +238,194 @@ __device__ __forceinline__ unsigned long long shfl_up_u64(unsigned long long v, 
     return ((unsigned long long)hi << 32) | lo;
 }
 
-__global__ void __launch_bounds__(kToppThreads) topp_count_kernel(const float *scores, int len, int skip0,
-                                                                 const float *extra0, float p, int cap,
-                                                                 int *count) {
-    __shared__ unsigned long long hmass[256];
-    __shared__ uint32_t hcnt[256];
-    __shared__ unsigned long long red[kToppThreads / 32];
-    __shared__ unsigned long long s_rem;
-    __shared__ uint32_t s_prefix, s_mask;
-    __shared__ int s_above, s_done, s_eq;
-    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+__global__ void __launch_bounds__(kChunkThreads) topp_total_kernel(const float *scores, int len, int skip0,
+                                                                  unsigned long long *total) {
+    __shared__ unsigned long long red[kChunkThreads / 32];
+    const int r = blockIdx.y, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const float *x = scores + (size_t)r * len;
-    const int first = skip0 ? 1 : 0;
-    // total mass of the candidates
+    const int c0 = max(blockIdx.x * kToppChunk, skip0), c1 = min(len, (int)(blockIdx.x + 1) * kToppChunk);
     unsigned long long part = 0;
-    for (int i = first + tid; i < len; i += kToppThreads) part += fixed_mass(__ldg(x + i));
+    for (int i = c0 + threadIdx.x; i < c1; i += kChunkThreads) part += fixed_mass(__ldg(x + i));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if (lane == 0) red[wid] = part;
     __syncthreads();
-    if (tid == 0) {
-        unsigned long long total = 0;
-        for (int w = 0; w < kToppThreads / 32; ++w) total += red[w];
-        const unsigned long long m0 = skip0 ? fixed_mass(extra0[r]) : 0ull;
-        unsigned long long target = (unsigned long long)ceil((double)p * (double)(total + m0));
-        target = min(target, total + m0);
-        s_rem = target > m0 ? target - m0 : 0ull;
-        s_prefix = 0u;
-        s_mask = 0u;
-        s_above = 0;
-        s_done = s_rem == 0ull;
-        s_eq = 0;
+    if (threadIdx.x == 0) {
+        unsigned long long t = 0;
+        for (int w = 0; w < kChunkThreads / 32; ++w) t += red[w];
+        atomicAdd(total + r, t);  // integer: the sum is exact in any order
+    }
+}
+
+__global__ void topp_init_kernel(const unsigned long long *total, int skip0, const float *extra0, float p,
+                                 ToppState *st, uint32_t *hcnt, unsigned long long *hmass) {
+    const int r = blockIdx.x;
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+        hcnt[(size_t)r * 256 + b] = 0u;
+        hmass[(size_t)r * 256 + b] = 0ull;
+    }
+    if (threadIdx.x == 0) {
+        const unsigned long long m0 = skip0 ? fixed_mass(extra0[r]) : 0ull, all = total[r] + m0;
+        unsigned long long target = (unsigned long long)ceil((double)p * (double)all);
+        target = min(target, all);
+        ToppState s;
+        s.prefix = 0u;
+        s.mask = 0u;
+        s.rem = target > m0 ? target - m0 : 0ull;
+        s.above = 0;
+        s.eq = 0;
+        s.done = s.rem == 0ull;
+        s.pad = 0;
+        st[r] = s;
+    }
+}
+
+__global__ void __launch_bounds__(kChunkThreads) topp_hist_kernel(const float *scores, int len, int skip0,
+                                                                 const ToppState *st, uint32_t *hcnt,
+                                                                 unsigned long long *hmass, int shift) {
+    __shared__ unsigned long long sm[256];
+    __shared__ uint32_t sc[256];
+    const int r = blockIdx.y, lane = threadIdx.x & 31;
+    const ToppState s = st[r];
+    if (s.done) return;
+    for (int b = threadIdx.x; b < 256; b += kChunkThreads) {
+        sm[b] = 0ull;
+        sc[b] = 0u;
     }
     __syncthreads();
-    for (int pass = 0; pass < 4 && !s_done; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int b = tid; b < 256; b += kToppThreads) {
-            hmass[b] = 0ull;
-            hcnt[b] = 0u;
+    const float *x = scores + (size_t)r * len;
+    const int c0 = max(blockIdx.x * kToppChunk, skip0), c1 = min(len, (int)(blockIdx.x + 1) * kToppChunk);
+    for (int i0 = c0; i0 < c1; i0 += kChunkThreads) {
+        const int i = i0 + threadIdx.x;
+        uint32_t u = 0u;
+        bool valid = false;
+        if (i < c1) {
+            u = __float_as_uint(__ldg(x + i));
+            valid = (u & s.mask) == s.prefix;
         }
-        __syncthreads();
-        const uint32_t prefix = s_prefix, pmask = s_mask;
-        for (int i0 = first; i0 < len; i0 += kToppThreads) {
-            const int i = i0 + tid;
-            uint32_t u = 0u;
-            bool valid = false;
-            if (i < len) {
-                u = __float_as_uint(__ldg(x + i));
-                valid = (u & pmask) == prefix;
+        const uint32_t bin = (u >> shift) & 255u;
+        const unsigned long long m = valid ? fixed_mass(__uint_as_float(u)) : 0ull;
+        // one shared atomic per distinct bin per warp: exact sums of <= 2^16 / 2^16 / 2^6 parts
+        unsigned todo = __ballot_sync(0xffffffffu, valid);
+        while (todo) {
+            const int leader = __ffs(todo) - 1;
+            const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+            const bool mine = valid && bin == lb;
+            const unsigned grp = __ballot_sync(0xffffffffu, mine);
+            const uint32_t a = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m & 0xffffu) : 0u);
+            const uint32_t b = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)((m >> 16) & 0xffffu) : 0u);
+            const uint32_t c = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m >> 32) : 0u);
+            if (lane == leader) {
+                atomicAdd(&sc[lb], (uint32_t)__popc(grp));
+                atomicAdd(&sm[lb], ((unsigned long long)c << 32) + ((unsigned long long)b << 16) + a);
             }
-            const uint32_t bin = (u >> shift) & 255u;
-            const unsigned long long m = valid ? fixed_mass(__uint_as_float(u)) : 0ull;
-            // one atomic per distinct bin per warp: exact sums of <= 2^16 / 2^16 / 2^6 parts
-            unsigned todo = __ballot_sync(0xffffffffu, valid);
-            while (todo) {
-                const int leader = __ffs(todo) - 1;
-                const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
-                const bool mine = valid && bin == lb;
-                const unsigned grp = __ballot_sync(0xffffffffu, mine);
-                const uint32_t a = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m & 0xffffu) : 0u);
-                const uint32_t b = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)((m >> 16) & 0xffffu) : 0u);
-                const uint32_t c = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m >> 32) : 0u);
-                if (lane == leader) {
-                    atomicAdd(&hcnt[lb], (uint32_t)__popc(grp));
-                    atomicAdd(&hmass[lb], ((unsigned long long)c << 32) + ((unsigned long long)b << 16) + a);
-                }
-                todo &= ~grp;
-            }
+            todo &= ~grp;
         }
-        __syncthreads();
-        if (wid == 0) {
-            // lane L owns bins 255-8L .. 248-8L; scan from the top for the bin where the mass is reached
-            unsigned long long ms[8], sum = 0;
-            uint32_t cs[8], csum = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                ms[e] = hmass[255 - 8 * lane - e];
-                cs[e] = hcnt[255 - 8 * lane - e];
-                sum += ms[e];
-                csum += cs[e];
-            }
-            unsigned long long incl = sum;
-            uint32_t cincl = csum;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const unsigned long long y = shfl_up_u64(incl, d);
-                const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, d);
-                if (lane >= d) {
-                    incl += y;
-                    cincl += cy;
-                }
-            }
-            const unsigned long long rem = s_rem;
-            unsigned long long cum = incl - sum;
-            uint32_t ccum = cincl - csum;
-            if (cum < rem && incl >= rem) {
-                int e = 0;
-                for (; e < 7; ++e) {
-                    if (cum + ms[e] >= rem) break;
-                    cum += ms[e];
-                    ccum += cs[e];
-                }
-                s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
-                s_mask = pmask | (255u << shift);
-                s_rem = rem - cum;
-                s_above += (int)ccum;
-                s_eq = (int)cs[e];
-            }
-        }
-        __syncthreads();
     }
-    if (tid == 0) {
-        int c = 0;
-        if (!s_done) {
-            // keys above the threshold, then as many of its ties (each of the same mass) as the rest needs
-            const unsigned long long mt = fixed_mass(__uint_as_float(s_prefix));
-            long long need = mt ? (long long)((s_rem + mt - 1) / mt) : (long long)s_eq;
-            need = min(need, (long long)s_eq);
-            c = s_above + (int)need;
+    __syncthreads();
+    for (int b = threadIdx.x; b < 256; b += kChunkThreads)
+        if (sc[b]) {
+            atomicAdd(hcnt + (size_t)r * 256 + b, sc[b]);
+            atomicAdd(hmass + (size_t)r * 256 + b, sm[b]);
         }
-        count[r] = min(c + (skip0 ? 1 : 0), cap);
+}
+
+// One warp per row: lane L owns bins 255-8L .. 248-8L; a scan from the top finds
+// the bin where the mass still needed is reached.  The histogram is cleared for
+// the next pass.
+__global__ void topp_digit_kernel(ToppState *st, uint32_t *hcnt, unsigned long long *hmass, int shift) {
+    const int r = blockIdx.x, lane = threadIdx.x;
+    ToppState s = st[r];
+    unsigned long long ms[8], sum = 0;
+    uint32_t cs[8], csum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const size_t at = (size_t)r * 256 + 255 - 8 * lane - e;
+        ms[e] = hmass[at];
+        cs[e] = hcnt[at];
+        hmass[at] = 0ull;
+        hcnt[at] = 0u;
+        sum += ms[e];
+        csum += cs[e];
     }
+    if (s.done) return;
+    unsigned long long incl = sum;
+    uint32_t cincl = csum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long y = shfl_up_u64(incl, d);
+        const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, d);
+        if (lane >= d) {
+            incl += y;
+            cincl += cy;
+        }
+    }
+    unsigned long long cum = incl - sum;
+    uint32_t ccum = cincl - csum;
+    if (cum < s.rem && incl >= s.rem) {
+        int e = 0;
+        for (; e < 7; ++e) {
+            if (cum + ms[e] >= s.rem) break;
+            cum += ms[e];
+            ccum += cs[e];
+        }
+        s.prefix |= (uint32_t)(255 - 8 * lane - e) << shift;
+        s.mask |= 255u << shift;
+        s.rem -= cum;
+        s.above += (int)ccum;
+        s.eq = (int)cs[e];
+        st[r] = s;
+    }
+}
+
+__global__ void topp_final_kernel(const ToppState *st, int skip0, int cap, int *count) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= gridDim.x * blockDim.x) return;
+    const ToppState s = st[r];
+    int c = 0;
+    if (!s.done) {
+        // keys above the threshold, then as many of its ties (each of the same mass) as the rest needs
+        const unsigned long long mt = fixed_mass(__uint_as_float(s.prefix));
+        long long need = mt ? (long long)((s.rem + mt - 1) / mt) : (long long)s.eq;
+        need = min(need, (long long)s.eq);
+        c = s.above + (int)need;
+    }
+    count[r] = min(c + skip0, cap);
 }
 
 }  // namespace
 
+size_t topp_scratch_bytes(int n_rows) {
+    return (size_t)n_rows * (sizeof(unsigned long long) + sizeof(ToppState) + 256 * (4 + 8)) + 1024;
+}
+
 cudaError_t run_topp_counts(const float *scores, int n_rows, int len, bool skip0, const float *extra0, float p,
-                            int cap, int *count, cudaStream_t st) {
+                            int cap, int *count, void *scratch, cudaStream_t st) {
     if (n_rows <= 0) return cudaSuccess;
-    topp_count_kernel<<<n_rows, kToppThreads, 0, st>>>(scores, len, skip0 ? 1 : 0, extra0, p, cap, count);
+    if (!scratch) return cudaErrorInvalidValue;
+    char *q = static_cast<char *>(scratch);
+    auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
+    size_t off = 0;
+    unsigned long long *total = reinterpret_cast<unsigned long long *>(q + off);
+    off = align(off + n_rows * sizeof(unsigned long long));
+    ToppState *state = reinterpret_cast<ToppState *>(q + off);
+    off = align(off + n_rows * sizeof(ToppState));
+    uint32_t *hcnt = reinterpret_cast<uint32_t *>(q + off);
+    off = align(off + (size_t)n_rows * 256 * sizeof(uint32_t));
+    unsigned long long *hmass = reinterpret_cast<unsigned long long *>(q + off);
+    const int sk = skip0 ? 1 : 0;
+    const int n_chunks = (len + kToppChunk - 1) / kToppChunk;
+    const dim3 grid(n_chunks, n_rows);
+    cudaError_t e = cudaMemsetAsync(total, 0, n_rows * sizeof(unsigned long long), st);
+    if (e != cudaSuccess) return e;
+    topp_total_kernel<<<grid, kChunkThreads, 0, st>>>(scores, len, sk, total);
+    topp_init_kernel<<<n_rows, 256, 0, st>>>(total, sk, extra0, p, state, hcnt, hmass);
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        topp_hist_kernel<<<grid, kChunkThreads, 0, st>>>(scores, len, sk, state, hcnt, hmass, shift);
+        topp_digit_kernel<<<n_rows, 32, 0, st>>>(state, hcnt, hmass, shift);
+    }
+    topp_final_kernel<<<n_rows, 1, 0, st>>>(state, sk, cap, count);
     return cudaGetLastError();
 }
 
