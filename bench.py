@@ -216,7 +216,14 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None):
             minf.minf_mixed_layer(q, k, v, pats, w.last_q, w.n_vertical, w.n_slash, w.topk, w.n_sink, w.window,
                                   scale, out=out, want_lse=False, ws=ws)
 
-        return (lambda: None), attend, ws, out, 0, 16
+        # launches per layer, by the pattern groups present
+        n_vs, n_bs = pats.count("vs"), pats.count("block")
+        topk_k = 1 if n <= 48 * 1024 else 12
+        per_batch = max(1, min(n_bs, (1 << 30) // ((n // 64) ** 2 * 4))) if n_bs else 1
+        launches = (4 + 2 * topk_k + 4) if n_vs else 0                            # estimate, top-k, plan, attention
+        launches += (2 + 2 * math.ceil(n_bs / per_batch) + 2) if n_bs else 0        # pool, scores + top-k, plan, attention
+        launches += sum(1 for p in ("ashape", "trishape", "dense") if p in pats)
+        return (lambda: None), attend, ws, out, 0, launches
     raise ValueError(w.pattern)
 
 

@@ -204,6 +204,23 @@ int check_scale(float scale) {
     return MINF_OK;
 }
 
+// One non-blocking side stream per device for the mixed layer, created on first use.
+cudaError_t side_stream(cudaStream_t *out) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev]) {
+        e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+        if (e != cudaSuccess) return e;
+    }
+    *out = streams[dev];
+    return cudaSuccess;
+}
+
 int check_ws(void *ws, size_t ws_bytes, size_t need) {
     if (!ws) return fail(MINF_ERR_INVALID, "null workspace");
     if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return fail(MINF_ERR_INVALID, "workspace not 256-byte aligned");
@@ -467,9 +484,9 @@ size_t minf_workspace_bytes(int op, int hq, int hkv, int n, int n_heads, int p1,
         c.take<int>((size_t)hq * p2);
         c.take<int>((size_t)hq * nb * p3);
         c.take<int>((size_t)hq * nb);
-        const size_t sub = std::max(std::max(bytes_vs_est(hkv, n, hq), bytes_vs_attn(n, hq, p1, p2)),
-                                    std::max(bytes_bs_est(hkv, n, hq), bytes_bs_attn(n, hq, p3)));
-        c.take<char>(sub);
+        // Vertical-Slash and Block-Sparse work run side by side: one scratch region each
+        c.take<char>(std::max(bytes_vs_est(hkv, n, hq), bytes_vs_attn(n, hq, p1, p2)));
+        c.take<char>(std::max(bytes_bs_est(hkv, n, hq), bytes_bs_attn(n, hq, p3)));
         return c.off;
     }
     }
@@ -670,37 +687,60 @@ int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v,
     int32_t *s_idx = c.take<int32_t>((size_t)hq * n_slash);
     int32_t *blk_idx = c.take<int32_t>((size_t)hq * nb * topk);
     int32_t *blk_cnt = c.take<int32_t>((size_t)hq * nb);
-    char *scratch = c.take<char>(0);
-    // estimates first (VS, then Block-Sparse), then the attention of every group
+    char *scratch_vs = c.take<char>(std::max(bytes_vs_est(hkv, n, hq), bytes_vs_attn(n, hq, n_vertical, n_slash)));
+    char *scratch_bs = c.take<char>(std::max(bytes_bs_est(hkv, n, hq), bytes_bs_attn(n, hq, topk)));
+    // Two streams (the caller's and a library side stream that starts after the
+    // work already queued on it): Vertical-Slash estimate and attention, then
+    // A-shape and Tri-shape on the caller's; Block-Sparse estimate and attention,
+    // then dense on the side stream, so each group's estimate overlaps the other
+    // group's attention.  The caller's stream waits for the side stream at the end.
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_side = nullptr;
+    const bool two = (sub[PAT_BLOCK].n_heads || sub[PAT_DENSE].n_heads) &&
+                     (sub[PAT_VS].n_heads || sub[PAT_ASHAPE].n_heads || sub[MINF_PATTERN_TRISHAPE].n_heads);
+    if (two) {
+        cudaError_t e = side_stream(&side);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_side, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_start, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_start, 0);
+        if (e != cudaSuccess) {
+            if (ev_start) cudaEventDestroy(ev_start);
+            if (ev_side) cudaEventDestroy(ev_side);
+            return cuda_fail(e, "side stream");
+        }
+    }
+    cudaStream_t st2 = two ? side : st;
+    int rc2 = MINF_OK;
     if (sub[PAT_VS].n_heads) {
-        rc = do_vs_estimate(sub[PAT_VS], q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws, scratch, st);
-        if (rc) return rc;
-        rc = do_vs_attention(sub[PAT_VS], q, k, v, scale, v_idx, n_vertical, s_idx, n_slash, out, lse, ws, scratch,
-                             true, st);
-        if (rc) return rc;
+        rc = do_vs_estimate(sub[PAT_VS], q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws, scratch_vs, st);
+        if (!rc)
+            rc = do_vs_attention(sub[PAT_VS], q, k, v, scale, v_idx, n_vertical, s_idx, n_slash, out, lse, ws,
+                                 scratch_vs, true, st);
     }
     if (sub[PAT_BLOCK].n_heads) {
-        rc = do_block_estimate(sub[PAT_BLOCK], q, k, topk, blk_idx, blk_cnt, scratch, st);
-        if (rc) return rc;
-        rc = do_block_attention(sub[PAT_BLOCK], q, k, v, scale, blk_idx, blk_cnt, topk, out, lse, ws, scratch, true,
-                                st);
-        if (rc) return rc;
+        rc2 = do_block_estimate(sub[PAT_BLOCK], q, k, topk, blk_idx, blk_cnt, scratch_bs, st2);
+        if (!rc2)
+            rc2 = do_block_attention(sub[PAT_BLOCK], q, k, v, scale, blk_idx, blk_cnt, topk, out, lse, ws,
+                                     scratch_bs, true, st2);
     }
-    if (sub[PAT_ASHAPE].n_heads) {
+    if (!rc && sub[PAT_ASHAPE].n_heads)
         rc = do_static_attention(PAT_ASHAPE, sub[PAT_ASHAPE], q, k, v, scale, n_sink, window, 0, out, lse, ws, true,
                                  st);
-        if (rc) return rc;
-    }
-    if (sub[MINF_PATTERN_TRISHAPE].n_heads) {
+    if (!rc && sub[MINF_PATTERN_TRISHAPE].n_heads)
         rc = do_static_attention(PAT_ASHAPE, sub[MINF_PATTERN_TRISHAPE], q, k, v, scale, n_sink, window, last_q, out,
                                  lse, ws, true, st);
-        if (rc) return rc;
+    if (!rc2 && sub[PAT_DENSE].n_heads)
+        rc2 = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, 0, out, lse, ws, true, st2);
+    if (two) {
+        // join even after a failed launch: nothing may stay queued behind the caller's back
+        cudaError_t e = cudaEventRecord(ev_side, side);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_side, 0);
+        cudaEventDestroy(ev_start);
+        cudaEventDestroy(ev_side);
+        if (e != cudaSuccess && !rc && !rc2) return cuda_fail(e, "side stream join");
     }
-    if (sub[PAT_DENSE].n_heads) {
-        rc = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, 0, out, lse, ws, true, st);
-        if (rc) return rc;
-    }
-    return MINF_OK;
+    return rc ? rc : rc2;
 }
 
 int minf_status(void *ws, minf_stream_t stream) {

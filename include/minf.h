@@ -221,7 +221,11 @@ int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16
  * minf_trishape_attention (n_sink, window, n_last = last_q), DENSE heads
  * minf_dense_attention.
  * out [hq][n][128] bf16, lse [hq][n] fp32 (nullable).  The indices are kept in
- * the workspace; everything runs on `stream`.
+ * the workspace.  VS, ASHAPE and TRISHAPE heads run on `stream`; BLOCK and
+ * DENSE heads run on a library side stream that starts after the work already
+ * queued on `stream`, so each group's estimate overlaps the other group's
+ * attention; `stream` waits for the side stream before anything queued after
+ * this call, so to the caller the whole layer is ordered on `stream`.
  */
 int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv,
                      int n, int d, float scale, const int8_t *head_pattern, int last_q,
