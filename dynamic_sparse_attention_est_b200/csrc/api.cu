@@ -270,6 +270,17 @@ void fill_attn_common(AttnParams &P, const Common &c, float scale, const void *k
         P.head_ids[i] = i < c.n_heads ? c.ids[i] : 0;
         P.out_slot[i] = i < c.n_heads ? (slot_is_id ? c.ids[i] : i) : 0;
     }
+    // group the listed heads by kv-head (stable), for the kv-head-major launch order
+    const int group = c.hq / c.hkv;
+    int ng = 0, pos = 0;
+    for (int g = 0; g < c.hkv; ++g) {
+        const int start = pos;
+        for (int i = 0; i < c.n_heads; ++i)
+            if (c.ids[i] / group == g) P.kv_order[pos++] = i;
+        if (pos > start) P.kv_start[ng++] = start;
+    }
+    P.kv_start[ng] = pos;
+    P.n_kvgroups = ng;
 }
 
 cudaError_t encode_attn_maps(AttnParams &P, const void *q, const void *k, const void *v, const Common &c) {

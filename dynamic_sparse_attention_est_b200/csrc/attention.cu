@@ -329,8 +329,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     auto bar = [&](int i) { return smem_u32(bars + i); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = P.n_qtiles - 1 - (int)(blockIdx.x / P.n_heads);  // heaviest tiles first
-    const int hp = (int)(blockIdx.x % P.n_heads);
+    // kv-head-major order; within a group the heaviest query tiles first, its heads side by side
+    int gi = 0;
+    while (gi + 1 < P.n_kvgroups && (int)blockIdx.x >= P.kv_start[gi + 1] * P.n_qtiles) ++gi;
+    const int gh = P.kv_start[gi + 1] - P.kv_start[gi];
+    const int local = (int)blockIdx.x - P.kv_start[gi] * P.n_qtiles;
+    const int t = P.n_qtiles - 1 - local / gh;
+    const int hp = P.kv_order[P.kv_start[gi] + local % gh];
     const int h = P.head_ids[hp];
     const int g = h / P.group;
     const int w_item = hp * P.n_qtiles + t;

@@ -73,6 +73,12 @@ struct AttnParams {
     int bit_words;
     int head_ids[MINF_MAX_HEADS];
     int out_slot[MINF_MAX_HEADS];  // output row block of each listed head (its position, or its id)
+    // Launch order: work items of one kv-head's listed q-heads are contiguous
+    // (query tiles heaviest first, the group's heads side by side), so the CTAs
+    // in flight share that kv-head's K and V in L2.
+    int n_kvgroups;
+    int kv_order[MINF_MAX_HEADS];       // head positions sorted by kv-head
+    int kv_start[MINF_MAX_HEADS + 1];   // kv_order index where each group starts
 };
 
 // Bits [start, start + 64) of a bitmap of nbits bits; positions outside
