@@ -48,6 +48,8 @@ __global__ void pool_kernel(const __nv_bfloat16 *x, const __grid_constant__ Head
     *reinterpret_cast<float4 *>(out + ((size_t)slot * nb + b) * kD + lane * 4) = res;
 }
 
+constexpr int kLd = 68;  // padded row of the transposed operand tiles (a multiple of 4 floats)
+
 // scores[hb][i][j] = Qp_i . Kp_j for one 64x64 tile of (i, j), j-tile <= i-tile.
 __global__ void __launch_bounds__(256) pooled_scores_kernel(const float *qp, const float *kp,
                                                             const __grid_constant__ HeadList hl, int group,
@@ -55,24 +57,28 @@ __global__ void __launch_bounds__(256) pooled_scores_kernel(const float *qp, con
     const int jt = blockIdx.x, it = blockIdx.y, hb = blockIdx.z;
     if (jt > it) return;
     extern __shared__ float sm[];
-    float *As = sm;              // [128][64] transposed pooled Q rows
-    float *Bs = sm + 128 * 64;   // [128][64] transposed pooled K rows
+    // pooled Q and K rows stored transposed, [128 d][kLd]: a warp stores a 4-row x 8-d
+    // patch, whose 32 words land in 32 different banks (4 d + row mod 32), and still
+    // reads whole 32-byte sectors from global memory
+    float *As = sm;
+    float *Bs = sm + kD * kLd;
     const int hp = hp0 + hb;
     const float *A = qp + (size_t)hp * nb * kD;
     const float *B = kp + (size_t)(hl.ids[hp] / group) * nb * kD;
-    for (int x = threadIdx.x; x < 64 * kD; x += 256) {
-        const int row = x / kD, d = x % kD;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int patch = warp; patch < (64 / 4) * (kD / 8); patch += 8) {
+        const int row = (patch / (kD / 8)) * 4 + (lane & 3), d = (patch % (kD / 8)) * 8 + (lane >> 2);
         const int gi = it * 64 + row, gj = jt * 64 + row;
-        As[d * 64 + row] = gi < nb ? A[(size_t)gi * kD + d] : 0.f;
-        Bs[d * 64 + row] = gj < nb ? B[(size_t)gj * kD + d] : 0.f;
+        As[d * kLd + row] = gi < nb ? A[(size_t)gi * kD + d] : 0.f;
+        Bs[d * kLd + row] = gj < nb ? B[(size_t)gj * kD + d] : 0.f;
     }
     __syncthreads();
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     float acc[4][4] = {};
 #pragma unroll 8
     for (int d = 0; d < kD; ++d) {
-        const float4 a = *reinterpret_cast<const float4 *>(As + d * 64 + ty * 4);
-        const float4 b = *reinterpret_cast<const float4 *>(Bs + d * 64 + tx * 4);
+        const float4 a = *reinterpret_cast<const float4 *>(As + d * kLd + ty * 4);
+        const float4 b = *reinterpret_cast<const float4 *>(Bs + d * kLd + tx * 4);
         const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -131,7 +137,7 @@ cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStrea
                                                    a.n, b.kp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int smem_scores = 2 * 128 * 64 * (int)sizeof(float);
+    const int smem_scores = 2 * kD * kLd * (int)sizeof(float);
     e = cudaFuncSetAttribute(pooled_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scores);
     if (e != cudaSuccess) return e;
     const int smem_row = nb * (int)sizeof(float);
