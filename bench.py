@@ -455,7 +455,11 @@ def main():
         b.record(s_up)
         torch.cuda.synchronize()
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-        e2e = {"value": a.elapsed_time(b) / e2e_steps, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            e2e_ms = shard.max_over_ranks(e2e_ms, device=dev)
+        # whole-job figure, like `value`: every rank ran e2e_steps layers
+        e2e = {"value": e2e_ms / (e2e_steps * world), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": host_out[0].numel() * host_out[0].element_size(),
                "steps": e2e_steps, "overlap": "upload, compute and download on separate streams"}
         del sets, x2
