@@ -329,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     auto bar = [&](int i) { return smem_u32(bars + i); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // kv-head-major order; within a group the heaviest query tiles first, its heads side by side
+    // groups of heads one after the other; within a group the heaviest query tiles first,
+    // its heads side by side
     int gi = 0;
     while (gi + 1 < P.n_kvgroups && (int)blockIdx.x >= P.kv_start[gi + 1] * P.n_qtiles) ++gi;
     const int gh = P.kv_start[gi + 1] - P.kv_start[gi];

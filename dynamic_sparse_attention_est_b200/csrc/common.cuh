@@ -73,9 +73,10 @@ struct AttnParams {
     int bit_words;
     int head_ids[MINF_MAX_HEADS];
     int out_slot[MINF_MAX_HEADS];  // output row block of each listed head (its position, or its id)
-    // Launch order: work items of one kv-head's listed q-heads are contiguous
-    // (query tiles heaviest first, the group's heads side by side), so the CTAs
-    // in flight share that kv-head's K and V in L2.
+    // Launch order: the listed heads in n_kvgroups groups, taken one group after
+    // the other; inside a group the heaviest query tiles first, its heads side by
+    // side.  Grouped by kv-head, the CTAs in flight share that kv-head's K and V
+    // in L2; a single group is the plain heaviest-first order.
     int n_kvgroups;
     int kv_order[MINF_MAX_HEADS];       // head positions sorted by kv-head
     int kv_start[MINF_MAX_HEADS + 1];   // kv_order index where each group starts
