@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--workload", default="vs-gqa-32k")
     ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--shard", default="layers", choices=["layers", "heads"],
+                    help="N > 1: one layer per rank (weak scaling), or the heads of one layer split over the "
+                         "ranks in whole GQA groups with an all-gather of the output (strong scaling)")
     ap.add_argument("--topp", type=float, default=None,
                     help="Vertical-Slash top-p budgets (p for verticals and slashes; the budgets become caps)")
     ap.add_argument("--vs-mode", default="exact", choices=["exact", "tiles"],
@@ -144,7 +147,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workload
-def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None):
+def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None, pats=None):
     """Returns (step(ws) -> out, attention-only call for timing, label of the attention call)."""
     q, k, v = x["q"], x["k"], x["v"]
     hq, hkv, n = w.hq, w.hkv, w.n
@@ -207,7 +210,7 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None):
 
         return (lambda: None), attend, ws, out, 0, 1
     if w.pattern == "mixed":
-        pats = synth.mixed_head_patterns(w, seed)
+        pats = pats if pats is not None else synth.mixed_head_patterns(w, seed)
         ws = minf.workspace(minf.workspace_bytes(minf.OP_MIXED_LAYER, hq, hkv, n, hq, w.n_vertical, w.n_slash,
                                                  w.topk), dev)
         out = torch.empty_like(q)
@@ -227,7 +230,7 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None):
     raise ValueError(w.pattern)
 
 
-def estimate_bytes(w) -> float:
+def estimate_bytes(w_run) -> float:
     """Algorithmic HBM bytes of one layer's index estimation (+ top-k), by pattern.
 
     Vertical-Slash: both passes stream K once per pair of q-heads sharing a
@@ -359,17 +362,43 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     from dynamic_sparse_attention_est_b200 import shard
 
-    seed = shard.rank_seed(args.seed, rank)
-    log(f"generating {w.name} on {dev}")
-    x = synth.generate(w, seed=seed, device=dev)
+    sharded = args.shard == "heads" and world > 1
+    parts, pats_local, w_run = None, None, w
+    if sharded:
+        # one layer, the same on every rank; this rank runs its whole GQA groups as a smaller layer
+        import dataclasses
+
+        if world > w.hkv:
+            raise SystemExit(f"--shard heads needs at most {w.hkv} ranks (one kv-head each)")
+        seed = args.seed
+        pats_all = synth.mixed_head_patterns(w, seed) if w.pattern == "mixed" else [w.pattern] * w.hq
+        parts = shard.partition_heads(pats_all, w.hkv, world)
+        mine = parts[rank]
+        grp = w.hq // w.hkv
+        kvs = sorted({h // grp for h in mine})
+        log(f"generating {w.name} on {dev}; this rank: q-heads {mine}")
+        xf = synth.generate(w, seed=seed, device=dev)
+        x = {"q": xf["q"][mine].contiguous(), "k": xf["k"][kvs].contiguous(), "v": xf["v"][kvs].contiguous()}
+        del xf
+        w_run = dataclasses.replace(w, hq=len(mine), hkv=len(kvs))
+        pats_local = [pats_all[h] for h in mine] if w.pattern == "mixed" else None
+        args.no_dense = True
+    else:
+        seed = shard.rank_seed(args.seed, rank)
+        log(f"generating {w.name} on {dev}")
+        x = synth.generate(w, seed=seed, device=dev)
     torch.cuda.synchronize()
     log("inputs ready")
-    estimate, attend, ws, out, n_est_k, n_att_k = make_step(w, x, torch, minf, synth, seed, args.vs_mode, args.topp)
+    estimate, attend_local, ws, out, n_est_k, n_att_k = make_step(w_run, x, torch, minf, synth, seed, args.vs_mode,
+                                                                  args.topp, pats_local)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        estimate()
-        attend()
+    if sharded:
+        def attend():
+            attend_local()
+            shard.gather_heads(out, parts, w.hq)  # the whole layer's output on every rank
+    else:
+        attend = attend_local
 
     for i in range(max(3, args.warmup)):
         estimate()
@@ -406,7 +435,8 @@ def main():
     if world > 1:
         elapsed = shard.max_over_ranks(elapsed, device=dev)
         dist.barrier()
-    ms_per_layer = elapsed / (args.steps * world)
+    layers_per_step = 1 if sharded else world  # whole-job layers finished per step
+    ms_per_layer = elapsed / (args.steps * layers_per_step)
     ms_per_step = elapsed / args.steps
 
     log(f"timed region done: {ms_per_layer:.3f} ms/layer")
@@ -419,7 +449,7 @@ def main():
         host_in = {key: x[key].cpu().pin_memory() for key in ("q", "k", "v")}
         x2 = {key: torch.empty_like(x[key]) for key in ("q", "k", "v")}
         sets = [(x, estimate, attend, out)]
-        e2, a2, _, o2, _, _ = make_step(w, x2, torch, minf, synth, seed, args.vs_mode, args.topp)
+        e2, a2, _, o2, _, _ = make_step(w_run, x2, torch, minf, synth, seed, args.vs_mode, args.topp, pats_local)
         sets.append((x2, e2, a2, o2))
         host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -459,7 +489,7 @@ def main():
         if world > 1:
             e2e_ms = shard.max_over_ranks(e2e_ms, device=dev)
         # whole-job figure, like `value`: every rank ran e2e_steps layers
-        e2e = {"value": e2e_ms / (e2e_steps * world), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": e2e_ms / (e2e_steps * layers_per_step), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": host_out[0].numel() * host_out[0].element_size(),
                "steps": e2e_steps, "overlap": "upload, compute and download on separate streams"}
         del sets, x2
@@ -511,7 +541,7 @@ def main():
         line = {
             "metric": METRIC, "value": round(ms_per_layer, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; RoPE'd N(0,1) with planted structure)",
             "config": {"workload": w.name, "pattern": w.pattern, "hq": w.hq, "hkv": w.hkv, "n": w.n,
                        "last_q": w.last_q, "n_vertical": w.n_vertical, "n_slash": w.n_slash, "topk": w.topk,
@@ -520,14 +550,16 @@ def main():
                        **({"budgets": f"top-p {args.topp} (n_vertical, n_slash as caps)"}
                           if w.pattern == "vs" and args.topp is not None else {}),
                        "l2": "inputs larger than L2 (no flush)",
-                       "parallelism": f"one layer per rank x{world}"},
+                       "parallelism": (f"heads of one layer over {world} ranks in whole GQA groups, "
+                                       f"output all-gathered (shards {[len(p) for p in parts]})") if sharded
+                       else f"one layer per rank x{world}"},
             "roofline": roofline,
             "attention_ms": round(attn_ms, 4),
             "estimate_ms": round(ms_per_step - attn_ms, 4),
-            "estimate_roofline": ({"bound": "hbm", "bytes": estimate_bytes(w),
-                                   "achieved": round(estimate_bytes(w) / ((ms_per_step - attn_ms) * 1e-3) / 1e9, 1),
+            "estimate_roofline": ({"bound": "hbm", "bytes": estimate_bytes(w_run),
+                                   "achieved": round(estimate_bytes(w_run) / ((ms_per_step - attn_ms) * 1e-3) / 1e9, 1),
                                    "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
-                                   "frac": round(estimate_bytes(w) / ((ms_per_step - attn_ms) * 1e-3) / 1e9
+                                   "frac": round(estimate_bytes(w_run) / ((ms_per_step - attn_ms) * 1e-3) / 1e9
                                                  / peaks.get("hbm_gbs"), 4)}
                                   if w.pattern in ("vs", "block") and ms_per_step > attn_ms else None),
             "computed_tiles": tiles, "mask_pairs": pairs,

@@ -1,9 +1,9 @@
 """The multi-rank path on CPU: two gloo ranks share the heads of one layer.
 
 Each rank attends its own shard of GQA groups (computed here with the fp64
-oracle standing in for the per-rank kernels), the shards are gathered, and the
-result must equal the single-process layer; the timing reduction returns the
-maximum over ranks.
+oracle standing in for the per-rank kernels), the shards are gathered with the
+padded all-gather the benchmark uses, and the result must equal the
+single-process layer; the timing reduction returns the maximum over ranks.
 """
 import os
 import socket
@@ -38,9 +38,7 @@ def _worker(rank, world, port, result_path):
     mine = parts[rank]
     orc = oracle.get()
     out, _ = orc.dense_attention(x["q"], x["k"], x["v"], 0.088, head_ids=mine)
-    full = torch.zeros(8, 256, 128, dtype=torch.float64)
-    full[mine] = torch.from_numpy(out)
-    dist.all_reduce(full)  # shards are disjoint: the sum assembles the layer
+    full = shard.gather_heads(torch.from_numpy(out), parts, 8)  # padded all-gather, head order restored
     t = shard.max_over_ranks(1.0 + rank)
     if rank == 0:
         ref, _ = orc.dense_attention(x["q"], x["k"], x["v"], 0.088)
@@ -76,3 +74,29 @@ def test_partition_is_balanced_and_keeps_groups_whole():
 
 def test_rank_seeds_differ():
     assert len({shard.rank_seed(0, r) for r in range(8)}) == 8
+
+
+def _gather_worker(rank, world, port, result_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # 4 GQA groups of 2 q-heads over 3 ranks: shards of unequal size
+    pats = ["vs", "vs", "block", "block", "ashape", "ashape", "dense", "dense"]
+    parts = shard.partition_heads(pats, 4, world)
+    local = torch.stack([torch.full((3, 5), float(h)) for h in parts[rank]]) if parts[rank] else torch.zeros(0, 3, 5)
+    full = shard.gather_heads(local, parts, 8)
+    if rank == 0:
+        np.save(result_path, np.array([full[h].eq(float(h)).all().item() for h in range(8)] +
+                                      [len(p) for p in parts]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_gather_heads_unequal_shards(tmp_path):
+    """Three ranks with shards of different sizes: the padded all-gather puts every head back in place."""
+    res = str(tmp_path / "gather.npy")
+    mp.start_processes(_gather_worker, args=(3, _free_port(), res), nprocs=3, join=True, start_method="spawn")
+    r = np.load(res)
+    assert r[:8].all()
+    sizes = r[8:].tolist()
+    assert sum(sizes) == 8 and max(sizes) != min(sizes), sizes  # the padding was exercised
