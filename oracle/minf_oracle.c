@@ -20,8 +20,8 @@
  *      the matrix product), keep the top-k key blocks of each query block.
  *   3. A-shape ([TALK] second observation; [NEWS] 方法介绍): a static mask of the
  *      first tokens plus a local window.  Tri-shape ([TALK], SCBench part, named
- *      only as an A-shape variant): this build reads it as the A-shape mask plus
- *      dense rows for the last queries.
+ *      only as an A-shape variant): read here as the A-shape mask plus dense
+ *      rows for the last queries.
  *   4. Masked-softmax attention over the key set each pattern selects, causal.
  *      Vertical-Slash has two key sets: token-exact (a key enters row i if it
  *      is a vertical or i - k is a selected offset) and whole slash tiles
@@ -486,7 +486,7 @@ int orc_ashape_attention(const float *q, const float *k, const float *v, int hq,
 }
 
 /* Tri-shape: A-shape plus dense rows for the last n_last queries (the reading
- * this build takes of the Tri-shape named in the AICon talk transcript
+ * taken here of the Tri-shape named in the AICon talk transcript
  * "以 KV 缓存为中心的高效长文本方法", SCBench part, as an A-shape variant). */
 int orc_trishape_attention(const float *q, const float *k, const float *v, int hq, int hkv, int n,
                            int d, double scale, const int *head_ids, int n_heads, int n_sink,
