@@ -420,18 +420,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             // tcgen05 issue: S(j) = Q K(j)^T into S[j % 2]; O[j % 2] += P(j) V(j) with P(j)
             // read from the first 64 columns of S[j % 2]; S(j + 2) is issued after P(j) V(j)
             // and the tensor pipe runs them in order, so P(j) is consumed before it is overwritten.
+            // step-0 descriptors of Q, K stage 0 and V stage 0; a stage adds its offset / 16
+            const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sV, 16384, 1024);
             auto issue_s = [&](int j) -> bool {
                 const int s = j % kStages;
                 if (!wait_bounded(bar(B_K_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j)))
                     return false;
                 tc_fence_after();
-                const uint32_t dS = tmem + (j & 1) * 128;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(dS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + s * kTileBytes + off, 16, 1024),
-                            kIdescQK, kk != 0);
-                }
+                umma_ss_tile(tmem + (j & 1) * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
                 umma_commit(bar(B_K_EMPTY + s));
                 umma_commit(bar(B_S_FULL + (j & 1)));
                 return true;
@@ -447,11 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (!wait_bounded(bar(B_P_FULL + b), (j >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j))) break;
                 if (!wait_bounded(bar(B_V_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j))) break;
                 tc_fence_after();
-                const uint32_t dO = tmem + 256 + b * 128, aP = tmem + b * 128;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(dO, aP + kk * 8, sdesc_sw128(sV + s * kTileBytes + kk * 2048, 16384, 1024), kIdescPV,
-                            (j >= 2 || kk > 0) ? 1u : 0u);
+                umma_ts_tile(tmem + 256 + b * 128, tmem + b * 128, dv0 + (uint64_t)((s * kTileBytes) >> 4), kIdescPV,
+                             j >= 2 ? 1u : 0u);
                 umma_commit(bar(B_V_EMPTY + s));
                 if (j + 2 < T && !issue_s(j + 2)) break;
             }

@@ -153,6 +153,55 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// One 128x128x128 tile as eight K = 16 steps in a single asm block (fewer
+// instructions for the issuing thread than eight separate calls).  a0/b0 are the
+// step-0 shared-memory descriptors of two K-major 128B-swizzled operands; step kk
+// sits 32 bytes further within a 64-element chunk and the second chunk 16 KB on,
+// i.e. +2 and +1024 in the descriptors' address field (16-byte units).  The first
+// step accumulates into D iff acc_first.
+__device__ __forceinline__ void umma_ss_tile(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                             uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %11, %12, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %13, %14, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %15, %16, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %17, %18, %3, t;\n\t}\n" ::"r"(d),
+        "l"(a0), "l"(b0), "r"(idesc), "r"(acc_first), "l"(a0 + 2), "l"(b0 + 2), "l"(a0 + 4), "l"(b0 + 4),
+        "l"(a0 + 6), "l"(b0 + 6), "l"(a0 + 1024), "l"(b0 + 1024), "l"(a0 + 1026), "l"(b0 + 1026),
+        "l"(a0 + 1028), "l"(b0 + 1028), "l"(a0 + 1030), "l"(b0 + 1030)
+        : "memory");
+}
+
+// The P.V tile: A = P from TMEM (a_tmem, 8 columns per K = 16 step), B = an
+// N-major 128B-swizzled operand whose step kk sits 2 KB further (+128 in the
+// descriptor).  The first step accumulates into D iff acc_first.
+__device__ __forceinline__ void umma_ts_tile(uint32_t d, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                             uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%11], %12, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%13], %14, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%15], %16, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%17], %18, %3, t;\n\t}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b0), "r"(idesc), "r"(acc_first), "r"(a_tmem + 8), "l"(b0 + 128), "r"(a_tmem + 16),
+        "l"(b0 + 256), "r"(a_tmem + 24), "l"(b0 + 384), "r"(a_tmem + 32), "l"(b0 + 512), "r"(a_tmem + 40),
+        "l"(b0 + 640), "r"(a_tmem + 48), "l"(b0 + 768), "r"(a_tmem + 56), "l"(b0 + 896)
+        : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
