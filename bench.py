@@ -230,7 +230,7 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None, pats=N
     raise ValueError(w.pattern)
 
 
-def estimate_bytes(w_run) -> float:
+def estimate_bytes(w) -> float:
     """Algorithmic HBM bytes of one layer's index estimation (+ top-k), by pattern.
 
     Vertical-Slash: both passes stream K once per pair of q-heads sharing a

@@ -1,0 +1,42 @@
+"""bench.py's host-side helpers on the CPU (argument parsing, work and byte counts).
+
+The timed path needs a GPU; these catch slips in the code around it that would
+otherwise only show on a GPU machine.
+"""
+import math
+import sys
+
+import pytest
+
+import bench
+from dynamic_sparse_attention_est_b200 import synth
+
+
+@pytest.mark.parametrize("name", sorted(synth.WORKLOADS))
+def test_estimate_bytes_per_workload(name):
+    w = synth.WORKLOADS[name]
+    b = bench.estimate_bytes(w)
+    if w.pattern in ("vs", "block"):
+        assert b > w.hkv * w.n * 256  # at least one read of K
+    else:
+        assert b == 0.0
+
+
+def test_parse_defaults_and_options(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse()
+    assert (a.gpus, a.workload, a.impl, a.vs_mode, a.shard, a.topp) == (1, "vs-gqa-32k", "minf", "exact", "layers", None)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--vs-mode", "tiles", "--topp", "0.9", "--shard", "heads"])
+    a = bench.parse()
+    assert (a.vs_mode, a.topp, a.shard) == ("tiles", 0.9, "heads")
+
+
+def test_traffic_only_for_the_captured_source():
+    assert bench.attention_traffic(None) is None
+    assert bench.attention_traffic("no-such-workload") is None
+    v = bench.attention_traffic("vs-gqa-32k")
+    assert v is None or v > 0
+
+
+def test_tile_flops():
+    assert bench.TILE_FLOPS == 4 * 128 ** 3 and math.isclose(bench.TILE_FLOPS / 1e6, 8.388608)
