@@ -69,7 +69,7 @@ def parse():
 # launch, from the ncu capture summarised in profiles/, valid only for the
 # attention source it was taken on (sha1 of csrc/attention.cu).
 TRAFFIC = {
-    "vs-gqa-32k": ("3cca896177f4967d9fc8cbe5f5bea358bca4d306", 3.521955e9 + 0.260125e9),
+    "vs-gqa-32k": ("a6b0491396fd96d54bf7d4ea0dc3a075ae57cf09", 5.434786e9 + 0.243624e9),
 }
 
 
