@@ -428,3 +428,44 @@ def test_vs_topp_then_attention(orc):
     out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
                                       scale=SCALE)
     check_attention(out, lse, ref, rl, "VS attention on top-p indices")
+
+
+def test_new_variants_on_an_unsorted_head_subset(orc):
+    """Whole slash tiles, top-p budgets and Block-Sparse on a listed, unsorted head subset
+    of a GQA layer with a ragged tail (n % 128 == 64)."""
+    n, hq, hkv = 448, 16, 4
+    q, k, v = inputs(n, hq, hkv, seed=28)
+    ids = [14, 1, 6, 9, 4]
+    qc, kc, vc = cuda(q, k, v)
+    vi, si = orc.vs_estimate(q, k, 40, 24, 36, SCALE, head_ids=ids)
+    ref, rl = orc.vs_tiles_attention(q, k, v, SCALE, vi, si, 128, head_ids=ids)
+    out, lse = minf.minf_vs_attention_tiles(qc, kc, vc, torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                            scale=SCALE, head_ids=ids)
+    check_attention(out, lse, ref, rl, "VS whole tiles, head subset")
+    tv, ts, tvc, tsc, vert, slash = orc.vs_estimate_topp(q, k, 40, 200, 200, 0.8, 0.6, SCALE, head_ids=ids,
+                                                         return_scores=True)
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(qc, kc, 40, 200, 200, 0.8, 0.6, scale=SCALE, head_ids=ids)
+    for p in range(len(ids)):
+        check_topp(gv[p].cpu().numpy(), gvc[p].item(), vert[p], 0.8, 200, False, f"top-p vertical subset {p}")
+        check_topp(gs[p].cpu().numpy(), gsc[p].item(), slash[p], 0.6, 200, True, f"top-p slash subset {p}")
+    bi, bc = orc.block_estimate(q, k, 64, 3, head_ids=ids)
+    gbi, gbc = minf.minf_block_estimate(qc, kc, topk=3, head_ids=ids)
+    ref, rl = orc.block_attention(q, k, v, SCALE, 64, bi, bc, head_ids=ids)
+    out, lse = minf.minf_block_attention(qc, kc, vc, torch.from_numpy(bi).cuda(), torch.from_numpy(bc).cuda(),
+                                         scale=SCALE, head_ids=ids)
+    check_attention(out, lse, ref, rl, "Block-Sparse head subset (kv-head-major launch)")
+
+
+def test_topp_p_one_and_tiny_p(orc):
+    """p = 1 with caps above n keeps (nearly) every key; a tiny p keeps one vertical and
+    offset 0 plus at most one more offset."""
+    n = 320
+    q, k, _ = inputs(n, 2, 1, seed=33)
+    qc, kc = cuda(q, k)
+    vi, si, vc, sc, vert, slash = orc.vs_estimate_topp(q, k, 64, n + 8, n + 8, 1.0, 1.0, SCALE, return_scores=True)
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(qc, kc, 64, n + 8, n + 8, 1.0, 1.0, scale=SCALE)
+    for p in range(2):
+        assert int(gvc[p]) >= n - 8 and int(gsc[p]) >= n - 8, "p = 1 keeps almost every key"
+        check_topp(gv[p].cpu().numpy(), gvc[p].item(), vert[p], 1.0, n + 8, False, "p = 1 vertical")
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(qc, kc, 64, 50, 50, 1e-6, 1e-6, scale=SCALE)
+    assert torch.all(gvc == 1) and torch.all(gsc <= 2) and torch.all(gs[:, 0] == 0)
