@@ -88,7 +88,11 @@ typedef struct CUstream_st *minf_stream_t; /* the same type as cudaStream_t */
  *   BLOCK_ESTIMATE, BLOCK_ATTENTION: p1 = topk
  *   MIXED_LAYER: p1 = n_vertical, p2 = n_slash, p3 = topk (n_heads ignored: all hq heads)
  *   others: unused.
- * Returns 0 for arguments the op would reject.
+ * Returns 0 for arguments the op would reject.  Growth: VS_ATTENTION keeps, per
+ * listed head and 128-query tile, the list of vertical keys that no slash range
+ * of the tile covers, so it needs about n_heads * (n / 128) * min(n_vertical, n)
+ * * 4 bytes (1 GiB for 32 heads at 1M tokens with 1000 verticals); the others
+ * grow as n_heads * n.  VS_ESTIMATE also serves minf_vs_estimate_topp.
  */
 size_t minf_workspace_bytes(int op, int hq, int hkv, int n, int n_heads, int p1, int p2, int p3);
 
