@@ -85,11 +85,12 @@ VsEstBufs carve_vs_est(Carver &c, int n, int n_heads, int n_pairs) {
 VsPlanBufs carve_vs_plan(Carver &c, int n, int n_heads, int n_vertical, int n_slash) {
     VsPlanBufs b{};
     b.words = n / 32;
+    b.stride = b.words + 2 * kBitGuard;
     b.vcap = std::min(n_vertical, n);
     b.scap = std::min(n_slash, n);
     const size_t nw = (size_t)n_heads * qtiles(n);
-    b.bits_v = c.take<uint32_t>((size_t)n_heads * b.words);
-    b.bits_s = c.take<uint32_t>((size_t)n_heads * b.words);
+    b.bits_v = c.take<uint32_t>((size_t)n_heads * b.stride) + kBitGuard;
+    b.bits_s = c.take<uint32_t>((size_t)n_heads * b.stride) + kBitGuard;
     b.vsorted = c.take<int>((size_t)n_heads * b.vcap);
     b.nvs = c.take<int>(n_heads);
     b.soff = c.take<int>((size_t)n_heads * b.scap);
@@ -367,7 +368,7 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
     P.vs_vstride = b.vcap;
     P.vs_bits_s = b.bits_s;
     P.vs_bits_v = b.bits_v;
-    P.bit_words = b.words;
+    P.bit_stride = b.stride;
     P.vs_tiles = tiles ? 1 : 0;
     e = run_attention(PAT_VS, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "vs attention launch");

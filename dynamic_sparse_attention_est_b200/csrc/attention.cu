@@ -119,6 +119,23 @@ struct TileGen {
 
     __device__ int tiles() const { return (total + 1) >> 1; }
 
+    // Moves past two halves without describing them (the other softmax
+    // warpgroup's tile): only Vertical-Slash keeps state beyond the count, and two
+    // slash halves inside the current group just advance its cursor.
+    __device__ void skip2(const AttnParams &P) {
+        if constexpr (PAT == PAT_VS) {
+            if (emitted + 2 <= nsh && cur_a + kHalf <= cur_b) {
+                emitted += 2;
+                cur_a += 2 * kHalf;
+            } else {
+                next(P);
+                next(P);
+            }
+        } else {
+            emitted += 2;
+        }
+    }
+
     __device__ HalfDesc next(const AttnParams &P) {
         HalfDesc h{HALF_EMPTY, 0, 0, 0};
         if (emitted >= total) {
@@ -186,8 +203,8 @@ struct TileGen {
     }
 };
 
-// Bitmap words a Vertical-Slash range half needs for one row; fetched one tile
-// ahead so that the loads' latency hides behind the current tile's softmax.
+// Bitmap words a Vertical-Slash range half needs for one row.  They are loaded
+// right after a softmax warpgroup hands over its P, while it waits for its next S.
 struct MaskWords {
     uint32_t s[3], v[3];
 };
@@ -198,12 +215,13 @@ __device__ __forceinline__ void mask_fetch(const AttnParams &P, const HalfDesc &
                                            MaskWords &mw) {
     if constexpr (PAT == PAT_VS) {
         if (h.kind != HALF_RANGE || P.vs_tiles) return;
-        const int ws0 = (q - h.ks - 63) >> 5, wv0 = h.ks >> 5;
+        // q - ks - 63 >= -190 (ks <= r0 + 127) and ks <= n - 1: the windows stay
+        // within the guard words on either side of the bitmaps
+        const uint32_t *ps = bits_s + ((q - h.ks - 63) >> 5), *pv = bits_v + (h.ks >> 5);
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
-            const int a = ws0 + i, b = wv0 + i;
-            mw.s[i] = (a >= 0 && a < P.bit_words) ? __ldg(bits_s + a) : 0u;
-            mw.v[i] = (b >= 0 && b < P.bit_words) ? __ldg(bits_v + b) : 0u;
+            mw.s[i] = __ldg(ps + i);
+            mw.v[i] = __ldg(pv + i);
         }
     }
 }
@@ -464,31 +482,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const float sl2 = P.scale_log2;
         const uint32_t *bits_s = nullptr, *bits_v = nullptr;
         if constexpr (PAT == PAT_VS) {
-            bits_s = P.vs_bits_s + (size_t)hp * P.bit_words;
-            bits_v = P.vs_bits_v + (size_t)hp * P.bit_words;
+            bits_s = P.vs_bits_s + (size_t)hp * P.bit_stride;
+            bits_v = P.vs_bits_v + (size_t)hp * P.bit_stride;
         }
         float m_run = -INFINITY, l_run = 0.f;
         unsigned long long pairs = 0;
         bool ok = true;
-        if (wg == 1) {  // tile 0 belongs to the other warpgroup
-            gen.next(P);
-            gen.next(P);
-        }
-        HalfDesc hd0 = gen.next(P), hd1 = gen.next(P);
-        MaskWords mw0, mw1;
-        mask_fetch<PAT>(P, hd0, q, bits_s, bits_v, mw0);
-        mask_fetch<PAT>(P, hd1, q, bits_s, bits_v, mw1);
+        if (wg == 1) gen.skip2(P);  // tile 0 belongs to the other warpgroup
+        // element masks of this warpgroup's next tile: described, their bitmap words
+        // loaded and combined while the warpgroup waits for that tile's S, so that
+        // only the two 64-bit masks stay live through the softmax
+        uint64_t mk0 = 0, mk1 = 0;
+        bool full = false;
+        auto prepare = [&]() {
+            const HalfDesc d0 = gen.next(P), d1 = gen.next(P);
+            MaskWords w0, w1;
+            mask_fetch<PAT>(P, d0, q, bits_s, bits_v, w0);
+            mask_fetch<PAT>(P, d1, q, bits_s, bits_v, w1);
+            mk0 = half_mask<PAT>(P, d0, q, r, vlist, w0);
+            mk1 = half_mask<PAT>(P, d1, q, r, vlist, w1);
+            full = (d0.flags & d1.flags & HF_FULL) != 0;  // uniform over the CTA
+        };
+        prepare();
         for (int j = wg; j < T; j += 2) {
-            // the next own tile (j + 2): descriptors now, its mask words in flight meanwhile
-            gen.next(P);  // the other warpgroup's tile j + 1
-            gen.next(P);
-            const HalfDesc nd0 = gen.next(P), nd1 = gen.next(P);
-            MaskWords nw0, nw1;
-            mask_fetch<PAT>(P, nd0, q, bits_s, bits_v, nw0);
-            mask_fetch<PAT>(P, nd1, q, bits_s, bits_v, nw1);
-            const uint64_t mk0 = half_mask<PAT>(P, hd0, q, r, vlist, mw0);
-            const uint64_t mk1 = half_mask<PAT>(P, hd1, q, r, vlist, mw1);
-            const bool full = (hd0.flags & hd1.flags & HF_FULL) != 0;  // uniform over the CTA
             if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
             const bool got = wait_bounded(bar(B_S_FULL + wg), (j >> 1) & 1, wc, wait_site(4 + wg, B_S_FULL + wg, j));
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // tcgen05.ld below is warp-wide
@@ -567,10 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar(B_P_FULL + wg));
-            hd0 = nd0;
-            hd1 = nd1;
-            mw0 = nw0;
-            mw1 = nw1;
+            gen.skip2(P);  // the other warpgroup's tile j + 1
+            prepare();     // tile j + 2
         }
         // ------------------------------------------------------------ epilogue
         ok = __all_sync(0xffffffffu, ok);
@@ -686,15 +700,15 @@ __global__ void bs_plan_kernel(const int *blk_idx, const int *blk_cnt, int topk,
 // Vertical-Slash: mark the index rows into per-head bitmaps (order-free,
 // duplicates merge, out-of-range entries ignored).
 __global__ void vs_mark_kernel(const int *v_idx, int n_vertical, const int *s_idx, int n_slash, int n,
-                               uint32_t *bits_v, uint32_t *bits_s, int words) {
+                               uint32_t *bits_v, uint32_t *bits_s, int stride) {
     const int hp = blockIdx.x;
     for (int i = threadIdx.x; i < n_vertical; i += blockDim.x) {
         const int x = v_idx[(size_t)hp * n_vertical + i];
-        if (x >= 0 && x < n) atomicOr(bits_v + (size_t)hp * words + (x >> 5), 1u << (x & 31));
+        if (x >= 0 && x < n) atomicOr(bits_v + (size_t)hp * stride + (x >> 5), 1u << (x & 31));
     }
     for (int i = threadIdx.x; i < n_slash; i += blockDim.x) {
         const int x = s_idx[(size_t)hp * n_slash + i];
-        if (x >= 0 && x < n) atomicOr(bits_s + (size_t)hp * words + (x >> 5), 1u << (x & 31));
+        if (x >= 0 && x < n) atomicOr(bits_s + (size_t)hp * stride + (x >> 5), 1u << (x & 31));
     }
 }
 
@@ -738,14 +752,15 @@ __device__ int block_extract_bits(const uint32_t *bm, int words, int *out, int c
 // one more than 128 short of its successor; the j-th start and the j-th end
 // bound group j.
 __global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint32_t *bits_v, const uint32_t *bits_s,
-                                                                     int words, int *vsorted, int *nvs, int vcap,
+                                                                     int words, int stride, int *vsorted, int *nvs,
+                                                                     int vcap,
                                                                      int *soff, int scap, int2 *groups,
                                                                      int *ngroups) {
     __shared__ TopkShared sh;
     const int hp = blockIdx.x;
-    const int cv = block_extract_bits<kExtractThreads>(bits_v + (size_t)hp * words, words,
+    const int cv = block_extract_bits<kExtractThreads>(bits_v + (size_t)hp * stride, words,
                                                        vsorted + (size_t)hp * vcap, vcap, sh);
-    const int cs = block_extract_bits<kExtractThreads>(bits_s + (size_t)hp * words, words,
+    const int cs = block_extract_bits<kExtractThreads>(bits_s + (size_t)hp * stride, words,
                                                        soff + (size_t)hp * scap, scap, sh);
     __syncthreads();  // the offsets written above are read by other threads below
     const int *so = soff + (size_t)hp * scap;
@@ -786,7 +801,7 @@ __device__ __forceinline__ bool any_bits(const uint32_t *bm, int lo, int hi) {
 // vertical keys that no slash range of this 128-row tile covers, and how many
 // of those precede the tile's first row (their halves need no element mask).
 __global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap, const int2 *groups,
-                                   const int *ngroups, int gstride, const uint32_t *bits_s, int words, int n,
+                                   const int *ngroups, int gstride, const uint32_t *bits_s, int stride, int n,
                                    int n_heads, int n_qtiles, int *nsh, int *nvert, int *nle, int *vlist) {
     const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -804,7 +819,7 @@ __global__ void vs_workitem_kernel(const int *vsorted, const int *nvs, int vcap,
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, s);
     const int *vs = vsorted + (size_t)hp * vcap;
-    const uint32_t *bs = bits_s + (size_t)hp * words;
+    const uint32_t *bs = bits_s + (size_t)hp * stride;
     int *dst = vlist + (size_t)w * vcap;
     const int cv = nvs[hp];
     int out = 0, le = 0;
@@ -889,15 +904,17 @@ cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_
 
 cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, const int *s_idx, int n_slash,
                         int n, int n_heads, int n_qtiles, cudaStream_t st) {
-    cudaError_t e = cudaMemsetAsync(b.bits_v, 0, sizeof(uint32_t) * (size_t)n_heads * b.words, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(b.bits_s, 0, sizeof(uint32_t) * (size_t)n_heads * b.words, st);
+    // the guards are cleared with the bitmaps
+    const size_t bytes = sizeof(uint32_t) * (size_t)n_heads * b.stride;
+    cudaError_t e = cudaMemsetAsync(b.bits_v - kBitGuard, 0, bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b.bits_s - kBitGuard, 0, bytes, st);
     if (e != cudaSuccess) return e;
-    vs_mark_kernel<<<n_heads, 256, 0, st>>>(v_idx, n_vertical, s_idx, n_slash, n, b.bits_v, b.bits_s, b.words);
-    vs_extract_kernel<<<n_heads, kExtractThreads, 0, st>>>(b.bits_v, b.bits_s, b.words, b.vsorted, b.nvs, b.vcap, b.soff,
-                                              b.scap, b.groups, b.ngroups);
+    vs_mark_kernel<<<n_heads, 256, 0, st>>>(v_idx, n_vertical, s_idx, n_slash, n, b.bits_v, b.bits_s, b.stride);
+    vs_extract_kernel<<<n_heads, kExtractThreads, 0, st>>>(b.bits_v, b.bits_s, b.words, b.stride, b.vsorted, b.nvs,
+                                                           b.vcap, b.soff, b.scap, b.groups, b.ngroups);
     const int nw = n_heads * n_qtiles;
     vs_workitem_kernel<<<(nw + 3) / 4, 128, 0, st>>>(b.vsorted, b.nvs, b.vcap, b.groups, b.ngroups, b.scap,
-                                                     b.bits_s, b.words, n, n_heads, n_qtiles, b.nsh, b.nvert,
+                                                     b.bits_s, b.stride, n, n_heads, n_qtiles, b.nsh, b.nvert,
                                                      b.nle, b.vlist);
     return cudaGetLastError();
 }

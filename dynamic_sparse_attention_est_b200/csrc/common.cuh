@@ -14,6 +14,10 @@ constexpr int kD = 128;        // head dimension
 constexpr int kTileM = 128;    // query rows per tile
 constexpr int kHalf = 64;      // keys per half-tile (a tile is two halves)
 constexpr int kBlock = 64;     // Block-Sparse block size / Vertical-Slash row granularity
+// Zero words on each side of a head's Vertical-Slash bitmap, so that a 64-bit
+// window starting up to 6 words before the first word or ending 2 words past the
+// last one reads zeros without a bounds check.
+constexpr int kBitGuard = 8;
 
 // Workspace header: status word + counters, first 256 bytes of every workspace.
 struct WsHeader {
@@ -68,9 +72,9 @@ struct AttnParams {
     const int *vs_nle;        // per work item: gathered keys at or before the tile's first row
     int vs_tiles;             // 1: slash ranges attended whole (causal mask only)
     int vs_vstride;
-    const uint32_t *vs_bits_s;  // per head: bitmap of slash offsets
+    const uint32_t *vs_bits_s;  // per head: bitmap of slash offsets (head hp at hp * bit_stride)
     const uint32_t *vs_bits_v;  // per head: bitmap of vertical keys
-    int bit_words;
+    int bit_stride;             // words per head, kBitGuard zero words on each side included
     int head_ids[MINF_MAX_HEADS];
     int out_slot[MINF_MAX_HEADS];  // output row block of each listed head (its position, or its id)
     // Launch order: the listed heads in n_kvgroups groups, taken one group after

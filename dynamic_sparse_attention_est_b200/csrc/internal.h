@@ -11,8 +11,8 @@ struct AttnParams;
 
 // Device buffers of the Vertical-Slash tile plan (all inside the workspace).
 struct VsPlanBufs {
-    uint32_t *bits_v, *bits_s;  // [n_heads][words]
-    int words;
+    uint32_t *bits_v, *bits_s;  // head hp's n bits at + hp * stride, kBitGuard zero words on each side
+    int words, stride;          // n / 32, words + 2 * kBitGuard
     int *vsorted, *nvs;         // [n_heads][vcap], [n_heads]
     int vcap;
     int *soff;                  // [n_heads][scap]
