@@ -523,13 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         if (!((mw >> e) & 1u)) sr[c][e] = 0xff800000u;  // -inf
                 }
             }
-            // row max over the 128 columns (three-input max)
-            float mx = -INFINITY;
+            // row max over the 128 columns: four independent three-input max chains
+            float mc[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c) {
+                mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
 #pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    mx = fmax3(mx, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                for (int e = 2; e < 32; e += 2)
+                    mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+            }
+            float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
             mx *= sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool want = m_new > m_run + 8.0f;  // includes m_run = -inf with a finite m_new
@@ -573,12 +576,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     else acc0 = f32x2_add(acc0, f32x2_pack(p0, p1));
                     pp[c >> 1][(c & 1) * 16 + e] = pack_bf16x2(p0, p1);
                 }
+                if (c == 1) tmem_st32(tS, pp[0]);  // P(j) columns 0-31 of S[wg], stored while 32-63 are computed
             }
             float a0, a1, b0, b1;
             f32x2_unpack(acc0, a0, a1);
             f32x2_unpack(acc1, b0, b1);
             l_run += (a0 + a1) + (b0 + b1);
-            tmem_st32(tS, pp[0]);       // P(j) over the first 64 columns of S[wg]
             tmem_st32(tS + 32, pp[1]);
             tmem_st_wait();
             tc_fence_before();
