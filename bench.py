@@ -69,7 +69,7 @@ def parse():
 # launch, from the ncu capture summarised in profiles/, valid only for the
 # attention source it was taken on (sha1 of csrc/attention.cu).
 TRAFFIC = {
-    "vs-gqa-32k": ("a6b0491396fd96d54bf7d4ea0dc3a075ae57cf09", 5.434786e9 + 0.243624e9),
+    "vs-gqa-32k": ("c6382aeec35c26373228da1d2479e8f6aa30cd76", 3.212797e9 + 0.236549e9),
 }
 
 
