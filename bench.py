@@ -174,9 +174,10 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None, pats=N
             vi, si = state["idx"]
             vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
 
-        # launches: 4 estimate kernels, two top-k rows (1 kernel up to 48K keys, else 12), top-p counts
-        topk_k = 1 if n <= 48 * 1024 else 12
-        return estimate, attend, ws, out, 4 + 2 * topk_k + (2 if topp is not None else 0), 4
+        # launches: 4 estimate kernels, top-k of both row sets (one kernel up to 48K keys,
+        # else 12 per row set), top-p counts (11 kernels per row set)
+        topk_launches = 1 if n <= 48 * 1024 else 24
+        return estimate, attend, ws, out, 4 + topk_launches + (22 if topp is not None else 0), 4
     if w.pattern == "block":
         ws_est = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ESTIMATE, hq, hkv, n, hq, w.topk), dev)
         ws = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ATTENTION, hq, hkv, n, hq, w.topk), dev)
@@ -221,9 +222,9 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None, pats=N
 
         # launches per layer, by the pattern groups present
         n_vs, n_bs = pats.count("vs"), pats.count("block")
-        topk_k = 1 if n <= 48 * 1024 else 12
+        topk_launches = 1 if n <= 48 * 1024 else 24
         per_batch = max(1, min(n_bs, (1 << 30) // ((n // 64) ** 2 * 4))) if n_bs else 1
-        launches = (4 + 2 * topk_k + 4) if n_vs else 0                            # estimate, top-k, plan, attention
+        launches = (4 + topk_launches + 4) if n_vs else 0                            # estimate, top-k, plan, attention
         launches += (2 + 2 * math.ceil(n_bs / per_batch) + 2) if n_bs else 0        # pool, scores + top-k, plan, attention
         launches += sum(1 for p in ("ashape", "trishape", "dense") if p in pats)
         return (lambda: None), attend, ws, out, 0, launches

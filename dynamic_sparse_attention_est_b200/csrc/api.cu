@@ -54,10 +54,11 @@ struct Carver {
 
 int qtiles(int n) { return (n + kTileM - 1) / kTileM; }
 
-// Vertical-Slash estimate: key chunking for about two CTAs per SM.
+// Vertical-Slash estimate: key chunking for one wave of one CTA per SM (148 SMs;
+// the kernel's shared memory allows one CTA per SM), whole chunks per head pair.
 void vs_est_geometry(int n, int n_pairs, int *n_chunks, int *chunk_tiles, int *n_ktiles) {
     const int kt = (n + 127) / 128;
-    int want = (296 + n_pairs - 1) / std::max(1, n_pairs);
+    int want = 148 / std::max(1, n_pairs);
     want = std::max(1, std::min(want, kt));
     const int ct = (kt + want - 1) / want;
     *n_ktiles = kt;

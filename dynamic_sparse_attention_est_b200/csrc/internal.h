@@ -93,6 +93,15 @@ cudaError_t run_wait_timeout_check(void *hdr, unsigned long long limit_ns, cudaS
 size_t topk_scratch_bytes(int n_rows, int len);
 cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
                           cudaStream_t st, const int *k_row = nullptr);
+// Two row sets of the same length (each with its own k, k_row and output) in
+// one launch when the rows fit the one-block path, else one after the other.
+struct TopkRows {
+    const float *scores;
+    int n_rows, k;
+    int *out;
+    const int *k_row;
+};
+cudaError_t run_topk_rows2(const TopkRows &a, const TopkRows &b, int len, void *scratch, cudaStream_t st);
 
 // Top-p counts (device, n_rows entries, each at most cap): the fewest keys of a
 // row, best first, whose scores reach p of the row's mass; with skip0 key 0 is

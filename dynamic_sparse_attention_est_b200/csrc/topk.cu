@@ -26,11 +26,16 @@ constexpr int kSmemRow = 48 * 1024;  // floats held in shared memory by the one-
 constexpr int kChunk = 8192;         // keys per block in the multi-block path
 constexpr int kChunkThreads = 256;
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_smem_kernel(const float *scores, int len, int k,
-                                                                      const int *k_row, int *out) {
+// One block per row; blocks [0, a.n_rows) take the rows of a, the rest those of b
+// (two independent row sets of the same length in one launch).
+__global__ void __launch_bounds__(kTopkThreads) topk_rows_smem_kernel(const TopkRows a, const TopkRows b, int len) {
     extern __shared__ float row[];
     __shared__ TopkShared sh;
-    const float *x = scores + (size_t)blockIdx.x * len;
+    const bool second = (int)blockIdx.x >= a.n_rows;
+    const int r = second ? (int)blockIdx.x - a.n_rows : (int)blockIdx.x;
+    const float *x = (second ? b.scores : a.scores) + (size_t)r * len;
+    const int k = second ? b.k : a.k;
+    const int *k_row = second ? b.k_row : a.k_row;
     for (int i = threadIdx.x * 4; i < len; i += kTopkThreads * 4) {
         if (i + 3 < len) {
             *reinterpret_cast<float4 *>(row + i) = __ldg(reinterpret_cast<const float4 *>(x + i));
@@ -39,8 +44,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_smem_kernel(const floa
         }
     }
     __syncthreads();
-    int *o = out + (size_t)blockIdx.x * k;
-    const int kr = k_row ? max(0, min(k_row[blockIdx.x], k)) : k;
+    int *o = (second ? b.out : a.out) + (size_t)r * k;
+    const int kr = k_row ? max(0, min(k_row[r], k)) : k;
     block_topk_ascending<kTopkThreads, false>(row, len, kr, o, 0, sh);
     for (int j = min(kr, len) + (int)threadIdx.x; j < k; j += kTopkThreads) o[j] = -1;
 }
@@ -435,16 +440,12 @@ size_t topk_scratch_bytes(int n_rows, int len) {
     return (size_t)n_rows * (sizeof(RowState) + 256 * sizeof(uint32_t) + 2 * (size_t)n_chunks * sizeof(int2)) + 1024;
 }
 
-cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
-                          cudaStream_t st, const int *k_row) {
-    if (n_rows <= 0 || k <= 0) return cudaSuccess;
-    if (len <= kSmemRow) {
-        const int smem = len * (int)sizeof(float);
-        cudaError_t e = cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        topk_rows_smem_kernel<<<n_rows, kTopkThreads, smem, st>>>(scores, len, k, k_row, out);
-        return cudaGetLastError();
-    }
+// Rows longer than kSmemRow: chunked radix select over many blocks.
+static cudaError_t run_topk_rows_long(const TopkRows &t, int len, void *scratch, cudaStream_t st) {
+    const float *scores = t.scores;
+    const int n_rows = t.n_rows, k = t.k;
+    const int *k_row = t.k_row;
+    int *out = t.out;
     if (!scratch) return cudaErrorInvalidValue;
     const int n_chunks = (len + kChunk - 1) / kChunk;
     char *p = static_cast<char *>(scratch);
@@ -468,6 +469,33 @@ cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *
     topk_offsets_kernel<<<n_rows, 32, 0, st>>>(state, cnt, offs, n_chunks);
     topk_write_kernel<<<grid, kChunkThreads, 0, st>>>(scores, len, k, state, offs, n_chunks, out);
     return cudaGetLastError();
+}
+
+cudaError_t run_topk_rows(const float *scores, int n_rows, int len, int k, int *out, void *scratch,
+                          cudaStream_t st, const int *k_row) {
+    return run_topk_rows2(TopkRows{scores, n_rows, k, out, k_row}, TopkRows{nullptr, 0, 0, nullptr, nullptr}, len,
+                          scratch, st);
+}
+
+cudaError_t run_topk_rows2(const TopkRows &a, const TopkRows &b, int len, void *scratch, cudaStream_t st) {
+    const TopkRows A = (a.n_rows > 0 && a.k > 0) ? a : TopkRows{nullptr, 0, 0, nullptr, nullptr};
+    const TopkRows B = (b.n_rows > 0 && b.k > 0) ? b : TopkRows{nullptr, 0, 0, nullptr, nullptr};
+    if (A.n_rows + B.n_rows == 0) return cudaSuccess;
+    if (len <= kSmemRow) {
+        const int smem = len * (int)sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        topk_rows_smem_kernel<<<A.n_rows + B.n_rows, kTopkThreads, smem, st>>>(A, B, len);
+        return cudaGetLastError();
+    }
+    if (!scratch) return cudaErrorInvalidValue;
+    // long rows: the row sets one after the other, sharing the scratch
+    for (const TopkRows *t : {&A, &B}) {
+        if (t->n_rows == 0) continue;
+        cudaError_t e = run_topk_rows_long(*t, len, scratch, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace minf

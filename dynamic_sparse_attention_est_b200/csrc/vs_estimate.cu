@@ -12,9 +12,11 @@
 //           offset 0 forced.
 // Both passes run S = Q K^T on the tensor cores: one CTA holds the last 64 rows
 // of two q-heads of the same kv-head as one M=128 tile (TMEM lanes 0-63 and
-// 64-127) and streams 128-key tiles of K through TMA.  Pass 2 reduces the
-// softmax weights through a skewed shared-memory buffer, so that column and
-// diagonal sums come out deterministic and without atomics.
+// 64-127) and streams 128-key tiles of K through TMA.  Pass 2 writes each
+// tile's softmax weights to a row-major shared-memory tile and sums it along
+// columns and along diagonals (both read patterns are bank-conflict-free), so
+// that the sums come out deterministic and without atomics.  The grid is one
+// wave of one CTA per SM: head pairs x key chunks.
 #include <cfloat>
 #include <cstring>
 
@@ -26,17 +28,17 @@ namespace minf {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 compute
 constexpr int kStages = 3;
 constexpr uint32_t kTileBytes = 32768;
 constexpr int kDiagW = 191;          // offsets one 128-key tile touches for 64 rows
-constexpr int kSkewRows = 95;        // offsets one 32-key chunk touches for 64 rows
-constexpr int kSkewStride = 65;      // padded row stride (floats) of the skew buffer
+// Row stride (floats) of the weight tile: rows start 16 bytes apart modulo the
+// 32 banks, so a warp's 16-byte row stores take the minimum four wavefronts.
+constexpr int kPStride = 132;
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kTileBytes;
-constexpr uint32_t kSmemSkew = kSmemK + kStages * kTileBytes;                 // 2*95*65 floats
-constexpr uint32_t kSmemDiag = kSmemSkew + 2 * kSkewRows * kSkewStride * 4;  // 2*191 floats
-constexpr uint32_t kSmemBar = (kSmemDiag + 2 * kDiagW * 4 + 255) & ~255u;
+constexpr uint32_t kSmemP = kSmemK + kStages * kTileBytes;  // 128 x kPStride floats
+constexpr uint32_t kSmemBar = (kSmemP + 128 * kPStride * 4 + 255) & ~255u;
 constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;
 
 enum : int { B_Q = 0, B_KF = 1, B_KE = 4, B_SF = 7, B_SE = 9, B_COUNT = 11 };
@@ -60,8 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_u32(smem) + kSmemQ, sK = smem_u32(smem) + kSmemK;
-    float *skew = reinterpret_cast<float *>(smem + kSmemSkew);
-    float *tdiag = reinterpret_cast<float *>(smem + kSmemDiag);
+    float *ptile = reinterpret_cast<float *>(smem + kSmemP);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + B_COUNT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT + 1);
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_SF + b), 1);
-            mbar_init(bar(B_SE + b), 128);
+            mbar_init(bar(B_SE + b), 256);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -140,7 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
             }
         }
     } else if (warp >= 4) {
-        const int r = threadIdx.x - 128;
+        // Eight compute warps: thread t holds columns [64 * half, 64 * half + 64) of
+        // row r (TMEM lane r: rows 0-63 are the first head's last 64 queries,
+        // rows 64-127 the second head's).
+        const int t = threadIdx.x - 128;
+        const int half = t >> 7, r = t & 127;
         const int rr = r & 63, hh = r >> 6;
         const int i = P.n - 64 + rr;  // query position of this row
         const bool head_ok = hh == 0 || pr.y >= 0;
@@ -155,80 +160,123 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
             const int b = j & 1;
             const int kt = kt0 + j;
             const bool got = wait_bounded(bar(B_SF + b), (j >> 1) & 1, wc, wait_site(7, B_SF + b, j));
-            // one decision for all 128 threads: the reduction below uses named barriers
-            if (named_bar_or(1, 128, !got || *abort_flag)) break;
+            // one decision for all compute threads: they meet at named barriers below
+            if (named_bar_or(1, 256, !got || *abort_flag)) break;
             tc_fence_after();
-            uint32_t sr[4][32];
+            uint32_t sr[2][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + b * 128 + c * 32, sr[c]);
+            for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_off + b * 128 + half * 64 + c * 32, sr[c]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+            for (int c = 0; c < 2; ++c) tmem_ld_wait(sr[c]);
             tc_fence_before();
             mbar_arrive(bar(B_SE + b));
-            const int cmax = row_ok ? i - kt * 128 : -1;  // columns c <= cmax are keys <= i
-            if constexpr (MODE == 0) {
-                float mx = -INFINITY;
+            // causal limit: columns c <= cmax are keys <= i (every column of the tiles
+            // below the last rows); rows outside the estimate take none
+            const int cmax = (row_ok ? i - kt * 128 : -1) - half * 64;
+            if (cmax < 63) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (c * 32 + e <= cmax) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-                mx *= sl2;
-                const float m_new = fmaxf(m_run, mx);
+                        if (c * 32 + e > cmax) sr[c][e] = 0xff800000u;  // -inf
+            }
+            if constexpr (MODE == 0) {
+                float mc[2];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+#pragma unroll
+                    for (int e = 2; e < 32; e += 2)
+                        mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                }
+                const float m_new = fmaxf(m_run, fmaxf(mc[0], mc[1]) * sl2);
                 if (m_new > -INFINITY) {
-                    float acc = 0.f;
+                    const uint64_t sl2x2 = f32x2_splat(sl2), negm = f32x2_splat(-m_new);
+                    uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c * 32 + e <= cmax)
-                                acc += ex2_approx(fmaf(__uint_as_float(sr[c][e]), sl2, -m_new));
-                    l_run = l_run * ex2_approx(m_run - m_new) + acc;
+                        for (int e = 0; e < 16; ++e) {
+                            float p0, p1;
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c][2 * e]),
+                                                              __uint_as_float(sr[c][2 * e + 1])),
+                                                   sl2x2, negm),
+                                         p0, p1);
+                            acc[e & 3] = f32x2_add(acc[e & 3], f32x2_pack(ex2_approx(p0), ex2_approx(p1)));
+                        }
+                    float a[8];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) f32x2_unpack(acc[u], a[2 * u], a[2 * u + 1]);
+                    const float tile_sum = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+                    l_run = l_run * ex2_approx(m_run - m_new) + tile_sum;
                     m_run = m_new;
                 }
             } else {
-                // zero this tile's diagonal accumulator
-                for (int x = r; x < 2 * kDiagW; x += 128) tdiag[x] = 0.f;
+                // normalised weights of this half row, then the whole tile in shared memory
+                named_bar_sync(1, 256);  // the previous tile's readers are done
+                float4 *dst = reinterpret_cast<float4 *>(ptile + r * kPStride + half * 64);
+                const uint64_t sl2x2 = f32x2_splat(sl2), negl = f32x2_splat(-lse2);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    named_bar_sync(1, 128);  // previous readers of the skew buffer are done
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float p = (cc * 32 + c <= cmax)
-                                            ? ex2_approx(fmaf(__uint_as_float(sr[cc][c]), sl2, -lse2))
-                                            : 0.f;
-                        skew[(hh * kSkewRows + (rr - c + 31)) * kSkewStride + rr] = p;
-                    }
-                    named_bar_sync(1, 128);
-                    for (int task = r; task < 64 + 2 * kSkewRows; task += 128) {
-                        if (task < 64) {  // column sum of one key over the 64 rows of one head
-                            const int h2 = task >> 5, c = task & 31;
-                            float s = 0.f;
-                            for (int r2 = 0; r2 < 64; ++r2) s += skew[(h2 * kSkewRows + (r2 - c + 31)) * kSkewStride + r2];
-                            const int key = kt * 128 + cc * 32 + c;
-                            const int hp2 = h2 == 0 ? pr.x : pr.y;
-                            if (hp2 >= 0 && key < P.n) P.vert[(size_t)hp2 * P.n + key] = s;
-                        } else {  // diagonal sum of one offset
-                            const int t2 = task - 64;
-                            const int h2 = t2 / kSkewRows, orel = t2 % kSkewRows;
-                            float s = 0.f;
-                            const int lo = max(0, orel - 31), hi = min(63, orel);
-                            for (int r2 = lo; r2 <= hi; ++r2) s += skew[(h2 * kSkewRows + orel) * kSkewStride + r2];
-                            tdiag[h2 * kDiagW + orel + 96 - 32 * cc] += s;
+                    for (int e = 0; e < 8; ++e) {
+                        float w[4];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float x0, x1;
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[c][4 * e + 2 * h2]),
+                                                              __uint_as_float(sr[c][4 * e + 2 * h2 + 1])),
+                                                   sl2x2, negl),
+                                         x0, x1);
+                            w[2 * h2] = ex2_approx(x0);
+                            w[2 * h2 + 1] = ex2_approx(x1);
                         }
+                        dst[c * 8 + e] = make_float4(w[0], w[1], w[2], w[3]);
                     }
-                }
-                named_bar_sync(1, 128);
-                for (int x = r; x < 2 * kDiagW; x += 128) {
-                    const int h2 = x / kDiagW;
+                named_bar_sync(1, 256);
+                // column sums: thread t owns key column t & 127 of head t >> 7 (a warp
+                // reads 32 consecutive floats of one row per step)
+                {
+                    const int h2 = t >> 7, c = t & 127;
+                    const float *col = ptile + h2 * 64 * kPStride + c;
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+                    for (int r2 = 0; r2 < 64; ++r2) acc[r2 & 7] += col[r2 * kPStride];
                     const int hp2 = h2 == 0 ? pr.x : pr.y;
-                    if (hp2 >= 0) P.diag[((size_t)hp2 * P.n_ktiles + kt) * kDiagW + (x % kDiagW)] = tdiag[x];
+                    const int key = kt * 128 + c;
+                    if (hp2 >= 0 && key < P.n)
+                        P.vert[(size_t)hp2 * P.n + key] =
+                            ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                 }
-                named_bar_sync(1, 128);
+                // diagonal sums: task u = (head, x), x = row - column + 127 in [0, 191),
+                // row rr in [x - 127, x] of that head; a warp takes 32 consecutive tasks,
+                // so each row read is 32 consecutive floats
+#pragma unroll 1
+                for (int u = t; u < 2 * kDiagW; u += 256) {
+                    const int h2 = u >= kDiagW ? 1 : 0, x = u - h2 * kDiagW;
+                    const float *base = ptile + h2 * 64 * kPStride + 127 - x;
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+                    for (int r2 = 0; r2 < 64; ++r2)
+                        if (r2 <= x && r2 >= x - 127) acc[r2 & 7] += base[r2 * (kPStride + 1)];
+                    const int hp2 = h2 == 0 ? pr.x : pr.y;
+                    if (hp2 >= 0)
+                        P.diag[((size_t)hp2 * P.n_ktiles + kt) * kDiagW + x] =
+                            ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+                }
             }
         }
         if constexpr (MODE == 0) {
-            P.part[((size_t)pair * P.n_chunks + chunk) * 128 + r] = make_float2(m_run, l_run);
+            // merge the two column halves of each row (the weight tile is unused in this pass)
+            float2 *xch = reinterpret_cast<float2 *>(ptile);
+            if (half == 1) xch[r] = make_float2(m_run, l_run);
+            named_bar_sync(1, 256);
+            if (half == 0) {
+                const float2 o = xch[r];
+                const float m = fmaxf(m_run, o.x);
+                const float l = m > -INFINITY ? l_run * ex2_approx(m_run - m) + o.y * ex2_approx(o.x - m) : 0.f;
+                P.part[((size_t)pair * P.n_chunks + chunk) * 128 + r] = make_float2(m, l);
+            }
         }
     }
     tc_fence_before();
@@ -335,9 +383,8 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
         kv = cv;
         ks = cs;
     }
-    e = run_topk_rows(b.vert, a.n_heads, a.n, a.n_vertical, a.v_idx, b.topk_scratch, st, kv);
-    if (e != cudaSuccess) return e;
-    return run_topk_rows(b.slash, a.n_heads, a.n, a.n_slash, a.s_idx, b.topk_scratch, st, ks);
+    return run_topk_rows2(TopkRows{b.vert, a.n_heads, a.n_vertical, a.v_idx, kv},
+                          TopkRows{b.slash, a.n_heads, a.n_slash, a.s_idx, ks}, a.n, b.topk_scratch, st);
 }
 
 }  // namespace minf
