@@ -47,7 +47,7 @@ TILE_FLOPS = 4 * 128 * 128 * 128  # QK^T and PV of one 128x128 tile, d = 128
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="vs-gqa-32k")
     ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
@@ -95,42 +95,52 @@ def measured_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region.
+
+    start() launches the sampler and waits for its first line, so that a slow
+    first NVML start does not leave the timed region without samples; mark()
+    and stop() bracket the timed region, and only samples that arrive between
+    them are kept (if the region is shorter than one interval, the first sample
+    after it stands in, and `samples` says how many were used)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (arrival time, text)
+        self.t_mark = None
 
-    def start(self):
+    def start(self, wait_s: float = 10.0):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.INTERVAL_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
             self.proc = None
+            return
+        t0 = time.monotonic()
+        while not self.lines and time.monotonic() - t0 < wait_s and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+    def mark(self):
+        self.t_mark = time.monotonic()
+
+    @staticmethod
+    def parse(lines):
+        """Median SM clock, max clock and the active throttle reasons of the sample lines."""
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -144,6 +154,23 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        t_end = time.monotonic()
+        # one more interval, so that a region shorter than the interval still gets the next sample
+        time.sleep(2 * self.INTERVAL_MS / 1000)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        t0 = self.t_mark if self.t_mark is not None else 0.0
+        inside = [ln for t, ln in self.lines if t0 <= t <= t_end]
+        if not inside:
+            inside = [ln for t, ln in self.lines if t > t_end][:1]
+        return self.parse(inside)
 
 
 # ----------------------------------------------------------------------------- workload
@@ -419,7 +446,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    time.sleep(0.3)
+    clocks.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)

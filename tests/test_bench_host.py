@@ -40,3 +40,12 @@ def test_traffic_only_for_the_captured_source():
 
 def test_tile_flops():
     assert bench.TILE_FLOPS == 4 * 128 ** 3 and math.isclose(bench.TILE_FLOPS / 1e6, 8.388608)
+
+
+def test_clock_lines_parse():
+    lines = ["1965, 1965, 700.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+             "1830, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+             "garbage"]
+    r = bench.ClockSampler.parse(lines)
+    assert r == {"sm_mhz": 1897.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert bench.ClockSampler.parse([])["samples"] == 0
