@@ -48,52 +48,80 @@ __global__ void pool_kernel(const __nv_bfloat16 *x, const __grid_constant__ Head
     *reinterpret_cast<float4 *>(out + ((size_t)slot * nb + b) * kD + lane * 4) = res;
 }
 
-constexpr int kLd = 68;  // padded row of the transposed operand tiles (a multiple of 4 floats)
+// Pooled-score tiles: 128 x 128 (i, j) per CTA, lower triangle only (the CTA's
+// index enumerates the tiles jt <= it), 256 threads with an 8 x 8 register
+// tile each (rows ty*4+u and 64+ty*4+u, columns tx*4+v and 64+tx*4+v), d in
+// chunks of 32 staged transposed in shared memory.  Per d step a thread reads
+// four 16-byte vectors for 64 FMAs, one byte per FMA: the shared-memory
+// bandwidth matches the fp32 FMA rate.
+constexpr int kSt = 128;        // tile edge
+constexpr int kDc = 32;         // d per stage
+constexpr int kLd = kSt + 4;    // padded row of the transposed tiles (4 mod 32 banks)
 
-// scores[hb][i][j] = Qp_i . Kp_j for one 64x64 tile of (i, j), j-tile <= i-tile.
 __global__ void __launch_bounds__(256) pooled_scores_kernel(const float *qp, const float *kp,
                                                             const __grid_constant__ HeadList hl, int group,
                                                             int hp0, int nb, float *scores) {
-    const int jt = blockIdx.x, it = blockIdx.y, hb = blockIdx.z;
-    if (jt > it) return;
-    extern __shared__ float sm[];
-    // pooled Q and K rows stored transposed, [128 d][kLd]: a warp stores a 4-row x 8-d
-    // patch, whose 32 words land in 32 different banks (4 d + row mod 32), and still
-    // reads whole 32-byte sectors from global memory
-    float *As = sm;
-    float *Bs = sm + kD * kLd;
+    // tile t of the lower triangle: it (it + 1) / 2 <= t < (it + 1) (it + 2) / 2
+    const int t = blockIdx.x, hb = blockIdx.y;
+    int it = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((it + 1) * (it + 2) / 2 <= t) ++it;
+    while (it * (it + 1) / 2 > t) --it;
+    const int jt = t - it * (it + 1) / 2;
+    __shared__ __align__(16) float As[kDc * kLd];
+    __shared__ __align__(16) float Bs[kDc * kLd];
     const int hp = hp0 + hb;
     const float *A = qp + (size_t)hp * nb * kD;
     const float *B = kp + (size_t)(hl.ids[hp] / group) * nb * kD;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int patch = warp; patch < (64 / 4) * (kD / 8); patch += 8) {
-        const int row = (patch / (kD / 8)) * 4 + (lane & 3), d = (patch % (kD / 8)) * 8 + (lane >> 2);
-        const int gi = it * 64 + row, gj = jt * 64 + row;
-        As[d * kLd + row] = gi < nb ? A[(size_t)gi * kD + d] : 0.f;
-        Bs[d * kLd + row] = gj < nb ? B[(size_t)gj * kD + d] : 0.f;
-    }
-    __syncthreads();
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-    float acc[4][4] = {};
-#pragma unroll 8
-    for (int d = 0; d < kD; ++d) {
-        const float4 a = *reinterpret_cast<const float4 *>(As + d * kLd + ty * 4);
-        const float4 b = *reinterpret_cast<const float4 *>(Bs + d * kLd + tx * 4);
-        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    float acc[8][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
-            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
+    for (int d0 = 0; d0 < kD; d0 += kDc) {
+        // a warp stores a 4-row x 8-d patch: its 32 words land in 32 different banks
+        // (4 d + row mod 32), and each row's 8 floats are one 32-byte sector in global memory
+        for (int patch = warp; patch < (kSt / 4) * (kDc / 8); patch += 8) {
+            const int row = (patch / (kDc / 8)) * 4 + (lane & 3), d = (patch % (kDc / 8)) * 8 + (lane >> 2);
+            const int gi = it * kSt + row, gj = jt * kSt + row;
+            As[d * kLd + row] = gi < nb ? A[(size_t)gi * kD + d0 + d] : 0.f;
+            Bs[d * kLd + row] = gj < nb ? B[(size_t)gj * kD + d0 + d] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int d = 0; d < kDc; ++d) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(As + d * kLd + ty * 4);
+            const float4 a1 = *reinterpret_cast<const float4 *>(As + d * kLd + 64 + ty * 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(Bs + d * kLd + tx * 4);
+            const float4 b1 = *reinterpret_cast<const float4 *>(Bs + d * kLd + 64 + tx * 4);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        }
+        __syncthreads();
     }
     float *S = scores + (size_t)hb * nb * nb;
+    const bool vec = (nb & 3) == 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int gi = it * 64 + ty * 4 + u;
+    for (int u = 0; u < 8; ++u) {
+        const int gi = it * kSt + (u >> 2) * 64 + ty * 4 + (u & 3);
         if (gi >= nb) continue;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const int gj = jt * 64 + tx * 4 + v;
-            if (gj < nb) S[(size_t)gi * nb + gj] = acc[u][v];
+        for (int h = 0; h < 2; ++h) {
+            const int gj = jt * kSt + h * 64 + tx * 4;
+            float *dst = S + (size_t)gi * nb + gj;
+            if (vec && gj + 3 < nb) {
+                *reinterpret_cast<float4 *>(dst) =
+                    make_float4(acc[u][4 * h], acc[u][4 * h + 1], acc[u][4 * h + 2], acc[u][4 * h + 3]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    if (gj + v < nb) dst[v] = acc[u][4 * h + v];
+            }
         }
     }
 }
@@ -137,17 +165,14 @@ cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStrea
                                                    a.n, b.kp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int smem_scores = 2 * kD * kLd * (int)sizeof(float);
-    e = cudaFuncSetAttribute(pooled_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scores);
-    if (e != cudaSuccess) return e;
     const int smem_row = nb * (int)sizeof(float);
     e = cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_row);
     if (e != cudaSuccess) return e;
-    const int tiles = (nb + 63) / 64;
+    const int tiles = (nb + kSt - 1) / kSt;
+    const int tri = tiles * (tiles + 1) / 2;
     for (int hp0 = 0; hp0 < a.n_heads; hp0 += b.head_batch) {
         const int hbn = min(b.head_batch, a.n_heads - hp0);
-        pooled_scores_kernel<<<dim3(tiles, tiles, hbn), 256, smem_scores, st>>>(b.qp, b.kp, hl, group, hp0, nb,
-                                                                               b.scores);
+        pooled_scores_kernel<<<dim3(tri, hbn), 256, 0, st>>>(b.qp, b.kp, hl, group, hp0, nb, b.scores);
         block_topk_kernel<<<dim3(nb, hbn), kRowThreads, smem_row, st>>>(b.scores, nb, a.topk, hp0, a.blk_idx,
                                                                        a.blk_cnt);
         e = cudaGetLastError();

@@ -81,11 +81,7 @@ __global__ void __launch_bounds__(kChunkThreads) topk_hist_kernel(const float *s
         const uint32_t u = in ? __float_as_uint(__ldg(x + i)) : 0u;
         const bool hit = in && (u & s.mask) == s.prefix;
         const uint32_t bin = (u >> shift) & 255u;
-        const uint32_t active = __ballot_sync(0xffffffffu, hit);
-        if (hit) {
-            const uint32_t peers = __match_any_sync(active, bin);
-            if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-        }
+        if (hit) atomicAdd(&h[bin], 1u);
     }
     __syncthreads();
     for (int b = threadIdx.x; b < 256; b += kChunkThreads)

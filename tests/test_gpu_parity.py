@@ -63,17 +63,18 @@ def test_block_attention_oracle_indices(orc, topk):
     check_attention(out, lse, ref, rl, f"block topk={topk}")
 
 
-def test_block_estimate_band(orc):
-    n = 2048
-    w = synth.Workload("t", "block", 4, 2, n, "clustered")
+@pytest.mark.parametrize("n,hq,hkv,topk", [(2048, 4, 2, 8),
+                                           (64 * 263, 2, 1, 100),    # several 128-block score tiles, nb % 4 != 0
+                                           (64 * 2100, 1, 1, 100)])  # rows longer than the warp-per-row limit
+def test_block_estimate_band(orc, n, hq, hkv, topk):
+    w = synth.Workload("t", "block", hq, hkv, n, "clustered")
     x = synth.generate(w, seed=1)
     q, k = x["q"], x["k"]
-    topk = 8
     bi, bc, _, _, sc = orc.block_estimate(q, k, 64, topk, return_scores=True)
     gi, gc = minf.minf_block_estimate(*cuda(q, k), topk=topk)
     gi, gc = gi.cpu().numpy(), gc.cpu().numpy()
     nb = n // 64
-    for hp in range(4):
+    for hp in range(hq):
         for i in range(nb):
             row = gi[hp, i, :gc[hp, i]]
             assert gc[hp, i] == min(topk, i + 1)
