@@ -85,6 +85,18 @@ def attention_traffic(workload: str):
     return entry[1] if sha == entry[0] else None
 
 
+def pick_bf16_peak(peaks, elapsed_ms, reasons):
+    """The bf16 denominator of the attention roofline and its key in the peaks file.
+
+    The burst figure (cuBLAS timed alone, clocks at their maximum) fits a timed
+    region shorter than a second that ran without power capping; the sustained
+    figure (a seconds-long loop under the 1 kW cap) fits a longer region, or
+    one during which the clock sampler saw sw_power_cap."""
+    sustained = elapsed_ms >= 1000.0 or "sw_power_cap" in (reasons or [])
+    key = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
+    return peaks.get(key), key
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -550,12 +562,12 @@ def main():
         del outd
 
     peaks, src = measured_peaks()
-    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    peak, peak_key = pick_bf16_peak(peaks, elapsed, clk.get("reasons"))
     achieved = tiles * TILE_FLOPS / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": attention_traffic(w.name if args.vs_mode == "exact" else None),
                 "kernel": "attn_kernel (timed with its plan kernels, CUDA events around the attention call)",
-                "peak_source": f"{src} bf16_tflops_sustained"}
+                "peak_source": f"{src} {peak_key} (timed region {elapsed:.0f} ms)"}
 
     log("dense comparison done")
     cpu = None

@@ -49,3 +49,11 @@ def test_clock_lines_parse():
     r = bench.ClockSampler.parse(lines)
     assert r == {"sm_mhz": 1897.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
     assert bench.ClockSampler.parse([])["samples"] == 0
+
+
+def test_bf16_peak_choice():
+    peaks = {"bf16_tflops": 1661.7, "bf16_tflops_sustained": 1406.6}
+    assert bench.pick_bf16_peak(peaks, 200.0, []) == (1661.7, "bf16_tflops")
+    assert bench.pick_bf16_peak(peaks, 200.0, ["sw_power_cap"]) == (1406.6, "bf16_tflops_sustained")
+    assert bench.pick_bf16_peak(peaks, 9000.0, []) == (1406.6, "bf16_tflops_sustained")
+    assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, 9000.0, []) == (1590.0, "bf16_tflops")
