@@ -52,8 +52,14 @@ def test_clock_lines_parse():
 
 
 def test_bf16_peak_choice():
-    peaks = {"bf16_tflops": 1661.7, "bf16_tflops_sustained": 1406.6}
-    assert bench.pick_bf16_peak(peaks, 200.0, []) == (1661.7, "bf16_tflops")
-    assert bench.pick_bf16_peak(peaks, 200.0, ["sw_power_cap"]) == (1406.6, "bf16_tflops_sustained")
-    assert bench.pick_bf16_peak(peaks, 9000.0, []) == (1406.6, "bf16_tflops_sustained")
-    assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, 9000.0, []) == (1590.0, "bf16_tflops")
+    peaks = {"bf16_tflops": 1661.7, "bf16_tflops_sustained": 1406.6, "sm_max_mhz": 1965.0,
+             "clocks_under_load": {"sm_mhz_median": 1350.0}}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    capped = {"sm_mhz": 1387.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.pick_bf16_peak(peaks, 200.0, full) == (1661.7, "bf16_tflops")
+    assert bench.pick_bf16_peak(peaks, 9000.0, capped) == (1406.6, "bf16_tflops_sustained")
+    # no clock record: the duration and the throttle reasons decide
+    assert bench.pick_bf16_peak(peaks, 200.0, {"sm_mhz": None, "reasons": []}) == (1661.7, "bf16_tflops")
+    assert bench.pick_bf16_peak(peaks, 200.0, {"sm_mhz": None, "reasons": ["sw_power_cap"]})[1] == "bf16_tflops_sustained"
+    assert bench.pick_bf16_peak(peaks, 9000.0, None)[1] == "bf16_tflops_sustained"
+    assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, 9000.0, capped) == (1590.0, "bf16_tflops")
