@@ -149,3 +149,41 @@ def test_mixed_1m_layer(orc):
         else:
             ref, rl = orc.ashape_attention(qh, kh, vh, SCALE, w.n_sink, w.window, rows=rows)
         check_attention(out[h, rows], lse[h, rows], ref[0], rl[0], f"mixed 1M head {h} ({p})")
+
+
+def test_trishape_128k_layer(orc):
+    """Tri-shape at the bench's size (n_last = last_q = 64 dense tail rows)."""
+    w = synth.WORKLOADS["trishape-gqa-128k"]
+    x = synth.generate(w, seed=0, device="cuda")
+    out, lse = minf.minf_trishape_attention(x["q"], x["k"], x["v"], w.n_sink, w.window, w.last_q, SCALE)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.n, 96)  # includes the last 64 rows, the dense tail
+    for h in (5, 26):
+        qh, kh, vh = head_inputs(x, h, w.hq // w.hkv)
+        ref, rl = orc.trishape_attention(qh, kh, vh, SCALE, w.n_sink, w.window, w.last_q, rows=rows)
+        check_attention(out[h, rows], lse[h, rows], ref[0], rl[0], f"Tri-shape 128K head {h}")
+
+
+def test_vs_32k_layer_topp(orc, vs32k):
+    """Top-p budgets (p = 0.95, the fixed budgets as caps) on the 32K layer: sampled
+    heads' sets are the shortest covers of the oracle's mass, and the attention on
+    them matches the oracle's."""
+    from parity import check_topp
+
+    w, x = vs32k
+    q, k, v = x["q"], x["k"], x["v"]
+    p = 0.95
+    gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(q, k, w.last_q, w.n_vertical, w.n_slash, p, p, SCALE)
+    out, lse = minf.minf_vs_attention(q, k, v, gv, gs, SCALE)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.n, 96)
+    grp = w.hq // w.hkv
+    for h in (3, 30):
+        qh, kh, vh = head_inputs(x, h, grp)
+        _, _, _, _, vert, slash = orc.vs_estimate_topp(qh, kh, w.last_q, w.n_vertical, w.n_slash, p, p, SCALE,
+                                                       return_scores=True)
+        check_topp(gv[h].cpu().numpy(), int(gvc[h]), vert[0], p, w.n_vertical, False, f"32K top-p vertical h{h}")
+        check_topp(gs[h].cpu().numpy(), int(gsc[h]), slash[0], p, w.n_slash, True, f"32K top-p slash h{h}")
+        ref, rl = orc.vs_attention(qh, kh, vh, SCALE, gv[h:h + 1].cpu().numpy(), gs[h:h + 1].cpu().numpy(),
+                                   rows=rows)
+        check_attention(out[h, rows], lse[h, rows], ref[0], rl[0], f"VS 32K top-p head {h}")

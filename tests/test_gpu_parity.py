@@ -470,3 +470,29 @@ def test_topp_p_one_and_tiny_p(orc):
         check_topp(gv[p].cpu().numpy(), gvc[p].item(), vert[p], 1.0, n + 8, False, "p = 1 vertical")
     gv, gs, gvc, gsc = minf.minf_vs_estimate_topp(qc, kc, 64, 50, 50, 1e-6, 1e-6, scale=SCALE)
     assert torch.all(gvc == 1) and torch.all(gsc <= 2) and torch.all(gs[:, 0] == 0)
+
+
+def test_repeat_runs_bit_identical():
+    """Estimates and attention are deterministic: no atomics decide a value (the
+    diagonal partials are added in a fixed order, each work item is one CTA), so
+    two runs on the same inputs, with other launches between them, agree bit for bit."""
+    n, hq, hkv = 4160, 4, 2
+    q, k, v = cuda(*inputs(n, hq, hkv, seed=7))
+    xb = synth.generate(synth.Workload("t", "block", hq, hkv, n, "clustered"), seed=7)
+    qb, kb, vb = cuda(xb["q"], xb["k"], xb["v"])
+
+    def once():
+        gv, gs = minf.minf_vs_estimate(q, k, last_q=64, n_vertical=200, n_slash=400, scale=SCALE)
+        o, l = minf.minf_vs_attention(q, k, v, gv, gs, scale=SCALE)
+        bi, bc = minf.minf_block_estimate(qb, kb, topk=20)
+        ob, lb = minf.minf_block_attention(qb, kb, vb, bi, bc, scale=SCALE)
+        torch.cuda.synchronize()
+        return [t.cpu() for t in (gv, gs, o, l, bi, bc, ob, lb)]
+
+    first = once()
+    minf.minf_dense_attention(qb, kb, vb, scale=SCALE)  # unrelated work between the two runs
+    second = once()
+    names = ["v_idx", "s_idx", "vs out", "vs lse", "blk_idx", "blk_cnt", "bs out", "bs lse"]
+    for name, a, b in zip(names, first, second):
+        assert torch.equal(a.view(torch.uint8) if a.dtype == torch.bfloat16 else a,
+                           b.view(torch.uint8) if b.dtype == torch.bfloat16 else b), f"{name} differs between runs"
