@@ -434,24 +434,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 for (int j = max(0, issued - kStages); j < issued; ++j)
                     wait_bounded(bar(full0 + j % kStages), (j / kStages) & 1, drain);
             }
-        } else if (warp == 1 && lane == 0 && T > 0) {
+        } else if (warp == 1 && T > 0) {
             // tcgen05 issue: S(j) = Q K(j)^T into S[j % 2]; O[j % 2] += P(j) V(j) with P(j)
             // read from the first 64 columns of S[j % 2]; S(j + 2) is issued after P(j) V(j)
             // and the tensor pipe runs them in order, so P(j) is consumed before it is overwritten.
+            // The whole warp runs this loop (waits, counters and descriptors stay warp-uniform,
+            // every decision is taken by the warp as one); elect.sync picks the lane that issues.
             // step-0 descriptors of Q, K stage 0 and V stage 0; a stage adds its offset / 16
             const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
             const uint64_t dv0 = sdesc_sw128(sV, 16384, 1024);
             auto issue_s = [&](int j) -> bool {
                 const int s = j % kStages;
-                if (!wait_bounded(bar(B_K_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j)))
-                    return false;
+                const bool got = wait_bounded(bar(B_K_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j));
+                if (!__all_sync(0xffffffffu, got)) return false;
                 tc_fence_after();
-                umma_ss_tile(tmem + (j & 1) * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
-                umma_commit(bar(B_K_EMPTY + s));
-                umma_commit(bar(B_S_FULL + (j & 1)));
+                umma_ss_tile_warp(tmem + (j & 1) * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
+                umma_commit_warp(bar(B_K_EMPTY + s));
+                umma_commit_warp(bar(B_S_FULL + (j & 1)));
                 return true;
             };
-            bool ok = wait_bounded(bar(B_Q_FULL), 0, wc, wait_site(3, B_Q_FULL, 0));
+            bool ok = __all_sync(0xffffffffu, wait_bounded(bar(B_Q_FULL), 0, wc, wait_site(3, B_Q_FULL, 0)));
             if (ok) {
                 tc_fence_after();
                 ok = issue_s(0);
@@ -459,16 +461,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             for (int j = 0; ok && j < T; ++j) {
                 const int b = j & 1, s = j % kStages;
-                if (!wait_bounded(bar(B_P_FULL + b), (j >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j))) break;
-                if (!wait_bounded(bar(B_V_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j))) break;
+                bool got = wait_bounded(bar(B_P_FULL + b), (j >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j));
+                if (!__all_sync(0xffffffffu, got)) break;
+                got = wait_bounded(bar(B_V_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j));
+                if (!__all_sync(0xffffffffu, got)) break;
                 tc_fence_after();
-                umma_ts_tile(tmem + 256 + b * 128, tmem + b * 128, dv0 + (uint64_t)((s * kTileBytes) >> 4), kIdescPV,
-                             j >= 2 ? 1u : 0u);
-                umma_commit(bar(B_V_EMPTY + s));
+                umma_ts_tile_warp(tmem + 256 + b * 128, tmem + b * 128, dv0 + (uint64_t)((s * kTileBytes) >> 4),
+                                  kIdescPV, j >= 2 ? 1u : 0u);
+                umma_commit_warp(bar(B_V_EMPTY + s));
                 if (j + 2 < T && !issue_s(j + 2)) break;
             }
-            umma_commit(bar(B_ALL_DONE));  // always close: the epilogue (or the abort path) waits on it
-            if (P.hdr) atomicAdd(&P.hdr->tiles, (unsigned long long)T);
+            umma_commit_warp(bar(B_ALL_DONE));  // always close: the epilogue (or the abort path) waits on it
+            if (P.hdr && lane == 0) atomicAdd(&P.hdr->tiles, (unsigned long long)T);
         }
     } else {
         // ---------------------------------------------------------- softmax warpgroups

@@ -202,6 +202,60 @@ __device__ __forceinline__ void umma_ts_tile(uint32_t d, uint32_t a_tmem, uint64
         : "memory");
 }
 
+// Warp-wide forms of umma_ss_tile / umma_ts_tile / umma_commit: every lane of a
+// converged warp calls them with the same (warp-uniform) operands and
+// elect.sync lets one lane issue, so the operands need not come from a
+// single-lane branch.
+__device__ __forceinline__ void umma_ss_tile_warp(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                                  uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %3, %3;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %11, %12, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %13, %14, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %15, %16, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %17, %18, %3, t;\n\t}\n" ::"r"(d),
+        "l"(a0), "l"(b0), "r"(idesc), "r"(acc_first), "l"(a0 + 2), "l"(b0 + 2), "l"(a0 + 4), "l"(b0 + 4),
+        "l"(a0 + 6), "l"(b0 + 6), "l"(a0 + 1024), "l"(b0 + 1024), "l"(a0 + 1026), "l"(b0 + 1026),
+        "l"(a0 + 1028), "l"(b0 + 1028), "l"(a0 + 1030), "l"(b0 + 1030)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_tile_warp(uint32_t d, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                                  uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %3, %3;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%11], %12, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%13], %14, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%15], %16, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%17], %18, %3, t;\n\t}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b0), "r"(idesc), "r"(acc_first), "r"(a_tmem + 8), "l"(b0 + 128), "r"(a_tmem + 16),
+        "l"(b0 + 256), "r"(a_tmem + 24), "l"(b0 + 384), "r"(a_tmem + 32), "l"(b0 + 512), "r"(a_tmem + 40),
+        "l"(b0 + 640), "r"(a_tmem + 48), "l"(b0 + 768), "r"(a_tmem + 56), "l"(b0 + 896)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
+        : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
