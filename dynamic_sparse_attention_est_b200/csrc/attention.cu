@@ -278,16 +278,10 @@ __device__ __forceinline__ void load_tile(uint32_t stage, uint32_t bar, const Ha
 #pragma unroll
     for (int s = 0; s < 2; ++s)
         if (hd[s].kind != HALF_GATHER) tma_bytes += 2 * 8192;
-    if (lane == 0) {
-        mbar_expect_tx(bar, tma_bytes);
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            if (hd[s].kind == HALF_GATHER) continue;
-            const int ks = hd[s].kind == HALF_RANGE ? hd[s].ks : 0;
-            tma_load_3d(stage + s * 8192, map, bar, 0, ks, g);
-            tma_load_3d(stage + 16384 + s * 8192, map, bar, 64, ks, g);
-        }
-    }
+    // the whole warp: warp-uniform operands, one elected lane adds the bytes and issues
+    const uint32_t halves = (hd[0].kind != HALF_GATHER ? 1u : 0u) | (hd[1].kind != HALF_GATHER ? 2u : 0u);
+    tma_load_stage_warp(stage, map, bar, tma_bytes, hd[0].kind == HALF_RANGE ? hd[0].ks : 0,
+                        hd[1].kind == HALF_RANGE ? hd[1].ks : 0, g, halves);
     bool gathered = false;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
@@ -405,14 +399,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const __nv_bfloat16 *raw = is_k ? P.k : P.v;
             const uint32_t stage0 = is_k ? sK : sV;
             const int full0 = is_k ? B_K_FULL : B_V_FULL, empty0 = is_k ? B_K_EMPTY : B_V_EMPTY;
-            if (is_k && lane == 0 && T > 0) {
+            if (is_k && T > 0) {
                 const int r0 = t * kTileM;
-                mbar_expect_tx(bar(B_Q_FULL), 4 * 8192);
-                tma_load_3d(sQ, &P.tmap_q, bar(B_Q_FULL), 0, r0, h);
-                tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q_FULL), 64, r0, h);
-                tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q_FULL), 0, r0 + 64, h);
-                tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q_FULL), 64, r0 + 64, h);
-                mbar_arrive(bar(B_Q_FULL));
+                tma_load_stage_warp(sQ, &P.tmap_q, bar(B_Q_FULL), 4 * 8192, r0, r0 + 64, h, 3u);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_Q_FULL));
             }
             int issued = 0;
             for (int j = 0; j < T; ++j) {

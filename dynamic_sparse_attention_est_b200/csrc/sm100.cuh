@@ -99,6 +99,34 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         "l"(tmap), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// Warp-wide load of a 128-row K or V stage (two 64-row halves, each two 64-column
+// boxes of a 3-D tensor map {128, n, heads}): every lane of a converged warp
+// calls it with the same operands, and one lane, picked by elect.sync, adds the
+// expected bytes to `bar` and issues the TMA loads of the halves flagged in
+// `halves` (bit 0: rows y0 into dst, bit 1: rows y1 into dst + 8192).  Callers
+// order their own arrive on `bar` after it with __syncwarp.
+__device__ __forceinline__ void tma_load_stage_warp(uint32_t dst, const void *tmap, uint32_t bar, uint32_t bytes,
+                                                    int y0, int y1, int z, uint32_t halves) {
+    asm volatile(
+        "{\n\t.reg .pred e, h0, h1;\n\t.reg .b32 f0, f1;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "and.b32 f0, %7, 1;\n\t"
+        "and.b32 f1, %7, 2;\n\t"
+        "setp.ne.and.b32 h0, f0, 0, e;\n\t"
+        "setp.ne.and.b32 h1, f1, 0, e;\n\t"
+        "@e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%2], %3;\n\t"
+        "@h0 cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {0, %4, %6}], [%2];\n\t"
+        "@h0 cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%8], [%1, {64, %4, %6}], [%2];\n\t"
+        "@h1 cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%9], [%1, {0, %5, %6}], [%2];\n\t"
+        "@h1 cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%10], [%1, {64, %5, %6}], [%2];\n\t}\n" ::"r"(dst),
+        "l"(tmap), "r"(bar), "r"(bytes), "r"(y0), "r"(y1), "r"(z), "r"(halves),
+        "r"(dst + 16384), "r"(dst + 8192), "r"(dst + 16384 + 8192)
+        : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }

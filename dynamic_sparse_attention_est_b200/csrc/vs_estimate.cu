@@ -99,45 +99,45 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
     const WaitCtl wc{abort_flag, P.status, P.wait_limit_ns};
 
     if (warp == 0) {
-        if (lane == 0 && T > 0) {
-            const int q0 = P.n - 64;
-            const int h1 = pr.y >= 0 ? pr.w : pr.z;
-            mbar_expect_tx(bar(B_Q), 4 * 8192);
-            tma_load_3d(sQ, &P.tmap_q, bar(B_Q), 0, q0, pr.z);
-            tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q), 64, q0, pr.z);
-            tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q), 0, q0, h1);
-            tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q), 64, q0, h1);
-            mbar_arrive(bar(B_Q));
+        if (T > 0) {
+            if (lane == 0) {
+                const int q0 = P.n - 64;
+                const int h1 = pr.y >= 0 ? pr.w : pr.z;
+                mbar_expect_tx(bar(B_Q), 4 * 8192);
+                tma_load_3d(sQ, &P.tmap_q, bar(B_Q), 0, q0, pr.z);
+                tma_load_3d(sQ + 16384, &P.tmap_q, bar(B_Q), 64, q0, pr.z);
+                tma_load_3d(sQ + 8192, &P.tmap_q, bar(B_Q), 0, q0, h1);
+                tma_load_3d(sQ + 16384 + 8192, &P.tmap_q, bar(B_Q), 64, q0, h1);
+                mbar_arrive(bar(B_Q));
+            }
+            // K tiles: the whole warp runs the loop (warp-uniform operands), one elected
+            // lane issues each stage's loads
             for (int j = 0; j < T; ++j) {
                 const int s = j % kStages;
-                if (!wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc, wait_site(5, B_KE + s, j))) break;
-                const uint32_t st = sK + s * kTileBytes;
+                const bool got = wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc, wait_site(5, B_KE + s, j));
+                if (!__all_sync(0xffffffffu, got)) break;
                 const int key0 = (kt0 + j) * 128;
-                mbar_expect_tx(bar(B_KF + s), kTileBytes);
-                tma_load_3d(st, &P.tmap_k, bar(B_KF + s), 0, key0, g);
-                tma_load_3d(st + 16384, &P.tmap_k, bar(B_KF + s), 64, key0, g);
-                tma_load_3d(st + 8192, &P.tmap_k, bar(B_KF + s), 0, key0 + 64, g);
-                tma_load_3d(st + 16384 + 8192, &P.tmap_k, bar(B_KF + s), 64, key0 + 64, g);
-                mbar_arrive(bar(B_KF + s));
+                tma_load_stage_warp(sK + s * kTileBytes, &P.tmap_k, bar(B_KF + s), kTileBytes, key0, key0 + 64, g, 3u);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_KF + s));
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && T > 0) {
-            bool ok = wait_bounded(bar(B_Q), 0, wc, wait_site(6, B_Q, 0));
+        if (T > 0) {
+            // the whole warp runs the issue loop; elect.sync picks the issuing lane
+            const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
+            bool ok = __all_sync(0xffffffffu, wait_bounded(bar(B_Q), 0, wc, wait_site(6, B_Q, 0)));
             if (ok) tc_fence_after();
             for (int j = 0; ok && j < T; ++j) {
                 const int s = j % kStages, b = j & 1;
-                if (!wait_bounded(bar(B_KF + s), (j / kStages) & 1, wc, wait_site(6, B_KF + s, j))) break;
-                if (!wait_bounded(bar(B_SE + b), ((j >> 1) & 1) ^ 1, wc, wait_site(6, B_SE + b, j))) break;
+                bool got = wait_bounded(bar(B_KF + s), (j / kStages) & 1, wc, wait_site(6, B_KF + s, j));
+                if (!__all_sync(0xffffffffu, got)) break;
+                got = wait_bounded(bar(B_SE + b), ((j >> 1) & 1) ^ 1, wc, wait_site(6, B_SE + b, j));
+                if (!__all_sync(0xffffffffu, got)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tmem + b * 128, sdesc_sw128(sQ + off, 16, 1024),
-                            sdesc_sw128(sK + s * kTileBytes + off, 16, 1024), kIdescQK, kk != 0);
-                }
-                umma_commit(bar(B_KE + s));
-                umma_commit(bar(B_SF + b));
+                umma_ss_tile_warp(tmem + b * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
+                umma_commit_warp(bar(B_KE + s));
+                umma_commit_warp(bar(B_SF + b));
             }
         }
     } else if (warp >= 4) {
