@@ -69,7 +69,7 @@ def parse():
 # launch, from the ncu capture summarised in profiles/, valid only for the
 # attention source it was taken on (sha1 of csrc/attention.cu).
 TRAFFIC = {
-    "vs-gqa-32k": ("c6382aeec35c26373228da1d2479e8f6aa30cd76", 3.212797e9 + 0.236549e9),
+    "vs-gqa-32k": ("022f5bbaac5dbbefb6cb9ff986b7b405095132b4", 3.272737e9 + 0.235946e9),
 }
 
 
