@@ -223,9 +223,10 @@ def make_step(w, x, torch, minf, synth, seed, vs_mode="exact", topp=None, pats=N
             vs_attention(q, k, v, vi, si, scale, out=out, want_lse=False, ws=ws)
 
         # launches: 4 estimate kernels, top-k of both row sets (one kernel up to 48K keys,
-        # else 12 per row set), top-p counts (11 kernels per row set)
+        # else 12 per row set), top-p counts (one kernel up to 48K keys, else 11 per row set)
         topk_launches = 1 if n <= 48 * 1024 else 24
-        return estimate, attend, ws, out, 4 + topk_launches + (22 if topp is not None else 0), 4
+        topp_launches = (1 if n <= 48 * 1024 else 22) if topp is not None else 0
+        return estimate, attend, ws, out, 4 + topk_launches + topp_launches, 4
     if w.pattern == "block":
         ws_est = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ESTIMATE, hq, hkv, n, hq, w.topk), dev)
         ws = minf.workspace(minf.workspace_bytes(minf.OP_BLOCK_ATTENTION, hq, hkv, n, hq, w.topk), dev)

@@ -110,5 +110,11 @@ cudaError_t run_topk_rows2(const TopkRows &a, const TopkRows &b, int len, void *
 size_t topp_scratch_bytes(int n_rows);
 cudaError_t run_topp_counts(const float *scores, int n_rows, int len, bool skip0, const float *extra0, float p,
                             int cap, int *count, void *scratch, cudaStream_t st);
+// Two row sets of the same length in one launch when the rows fit the
+// one-block path (same counts as run_topp_counts), else one after the other.
+cudaError_t run_topp_counts2(const float *scores_a, int n_rows_a, bool skip0_a, const float *extra0_a, float p_a,
+                             int cap_a, int *count_a, const float *scores_b, int n_rows_b, bool skip0_b,
+                             const float *extra0_b, float p_b, int cap_b, int *count_b, int len, void *scratch,
+                             cudaStream_t st);
 
 }  // namespace minf

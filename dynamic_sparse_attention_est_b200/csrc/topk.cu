@@ -394,7 +394,176 @@ __global__ void topp_final_kernel(const ToppState *st, int skip0, int cap, int *
     count[r] = min(c + skip0, cap);
 }
 
+// Rows of up to kSmemRow floats: one 1024-thread block per row does the whole
+// top-p count (total, four mass-histogram digit passes, final count) with the
+// row in shared memory, and blocks [0, a.n_rows) take row set a, the rest row
+// set b.  The arithmetic is that of the multi-block kernels above: the same
+// fixed-point masses, exact integer sums, the same digit search and final count.
+struct ToppRows {
+    const float *scores;
+    int n_rows, skip0, cap;
+    const float *extra0;
+    float p;
+    int *count;
+};
+
+__global__ void __launch_bounds__(kTopkThreads) topp_rows_smem_kernel(const ToppRows a, const ToppRows b, int len) {
+    extern __shared__ float row[];
+    __shared__ unsigned long long hm[256];
+    __shared__ uint32_t hc[256];
+    __shared__ unsigned long long red[kTopkThreads / 32];
+    __shared__ ToppState sst;
+    const bool second = (int)blockIdx.x >= a.n_rows;
+    const ToppRows &g = second ? b : a;
+    const int r = second ? (int)blockIdx.x - a.n_rows : (int)blockIdx.x;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const float *x = g.scores + (size_t)r * len;
+    for (int i = threadIdx.x * 4; i < len; i += kTopkThreads * 4) {
+        if (i + 3 < len) {
+            *reinterpret_cast<float4 *>(row + i) = __ldg(reinterpret_cast<const float4 *>(x + i));
+        } else {
+            for (int j = i; j < len; ++j) row[j] = x[j];
+        }
+    }
+    __syncthreads();
+    // total mass of the keys from skip0 on (exact: integer sums)
+    unsigned long long part = 0;
+    for (int i = g.skip0 + (int)threadIdx.x; i < len; i += kTopkThreads) part += fixed_mass(row[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) red[wid] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long total = 0;
+        for (int w = 0; w < kTopkThreads / 32; ++w) total += red[w];
+        const unsigned long long m0 = g.skip0 ? fixed_mass(g.extra0[r]) : 0ull, all = total + m0;
+        unsigned long long target = (unsigned long long)ceil((double)g.p * (double)all);
+        target = min(target, all);
+        ToppState st0;
+        st0.prefix = 0u;
+        st0.mask = 0u;
+        st0.rem = target > m0 ? target - m0 : 0ull;
+        st0.above = 0;
+        st0.eq = 0;
+        st0.done = st0.rem == 0ull;
+        st0.pad = 0;
+        sst = st0;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const ToppState s = sst;
+        if (s.done) break;  // uniform: every thread read the same state
+        const int shift = 24 - 8 * pass;
+        for (int bb = threadIdx.x; bb < 256; bb += kTopkThreads) {
+            hm[bb] = 0ull;
+            hc[bb] = 0u;
+        }
+        __syncthreads();
+        for (int i0 = g.skip0; i0 < len; i0 += kTopkThreads) {
+            const int i = i0 + threadIdx.x;
+            uint32_t u = 0u;
+            bool valid = false;
+            if (i < len) {
+                u = __float_as_uint(row[i]);
+                valid = (u & s.mask) == s.prefix;
+            }
+            const uint32_t bin = (u >> shift) & 255u;
+            const unsigned long long m = valid ? fixed_mass(__uint_as_float(u)) : 0ull;
+            // one shared atomic per distinct bin per warp: exact sums of <= 2^16 / 2^16 / 2^6 parts
+            unsigned todo = __ballot_sync(0xffffffffu, valid);
+            while (todo) {
+                const int leader = __ffs(todo) - 1;
+                const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+                const bool mine = valid && bin == lb;
+                const unsigned grp = __ballot_sync(0xffffffffu, mine);
+                const uint32_t a0 = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m & 0xffffu) : 0u);
+                const uint32_t a1 = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)((m >> 16) & 0xffffu) : 0u);
+                const uint32_t a2 = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)(m >> 32) : 0u);
+                if (lane == leader) {
+                    atomicAdd(&hc[lb], (uint32_t)__popc(grp));
+                    atomicAdd(&hm[lb], ((unsigned long long)a2 << 32) + ((unsigned long long)a1 << 16) + a0);
+                }
+                todo &= ~grp;
+            }
+        }
+        __syncthreads();
+        if (wid == 0) {
+            // lane L owns bins 255-8L .. 248-8L; a scan from the top finds the bin where
+            // the mass still needed is reached
+            unsigned long long ms[8], sum = 0;
+            uint32_t cs[8], csum = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ms[e] = hm[255 - 8 * lane - e];
+                cs[e] = hc[255 - 8 * lane - e];
+                sum += ms[e];
+                csum += cs[e];
+            }
+            unsigned long long incl = sum;
+            uint32_t cincl = csum;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const unsigned long long y = shfl_up_u64(incl, d);
+                const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, d);
+                if (lane >= d) {
+                    incl += y;
+                    cincl += cy;
+                }
+            }
+            unsigned long long cum = incl - sum;
+            uint32_t ccum = cincl - csum;
+            if (cum < s.rem && incl >= s.rem) {
+                int e = 0;
+                for (; e < 7; ++e) {
+                    if (cum + ms[e] >= s.rem) break;
+                    cum += ms[e];
+                    ccum += cs[e];
+                }
+                ToppState n = s;
+                n.prefix |= (uint32_t)(255 - 8 * lane - e) << shift;
+                n.mask |= 255u << shift;
+                n.rem -= cum;
+                n.above += (int)ccum;
+                n.eq = (int)cs[e];
+                sst = n;
+            }
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const ToppState s = sst;
+        int c = 0;
+        if (!s.done) {
+            // keys above the threshold, then as many of its ties (each of the same mass) as the rest needs
+            const unsigned long long mt = fixed_mass(__uint_as_float(s.prefix));
+            long long need = mt ? (long long)((s.rem + mt - 1) / mt) : (long long)s.eq;
+            need = min(need, (long long)s.eq);
+            c = s.above + (int)need;
+        }
+        g.count[r] = min(c + g.skip0, g.cap);
+    }
+}
+
 }  // namespace
+
+cudaError_t run_topp_counts2(const float *scores_a, int n_rows_a, bool skip0_a, const float *extra0_a, float p_a,
+                             int cap_a, int *count_a, const float *scores_b, int n_rows_b, bool skip0_b,
+                             const float *extra0_b, float p_b, int cap_b, int *count_b, int len, void *scratch,
+                             cudaStream_t st) {
+    if (len <= kSmemRow && n_rows_a + n_rows_b > 0) {
+        const int smem = len * (int)sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(topp_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const ToppRows A{scores_a, max(n_rows_a, 0), skip0_a ? 1 : 0, cap_a, extra0_a, p_a, count_a};
+        const ToppRows B{scores_b, max(n_rows_b, 0), skip0_b ? 1 : 0, cap_b, extra0_b, p_b, count_b};
+        topp_rows_smem_kernel<<<A.n_rows + B.n_rows, kTopkThreads, smem, st>>>(A, B, len);
+        return cudaGetLastError();
+    }
+    cudaError_t e = run_topp_counts(scores_a, n_rows_a, len, skip0_a, extra0_a, p_a, cap_a, count_a, scratch, st);
+    if (e != cudaSuccess) return e;
+    return run_topp_counts(scores_b, n_rows_b, len, skip0_b, extra0_b, p_b, cap_b, count_b, scratch, st);
+}
 
 size_t topp_scratch_bytes(int n_rows) {
     return (size_t)n_rows * (sizeof(unsigned long long) + sizeof(ToppState) + 256 * (4 + 8)) + 1024;

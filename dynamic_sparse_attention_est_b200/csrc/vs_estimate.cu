@@ -374,11 +374,8 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
     if (a.topp) {
         // top-p: per-row counts by mass, then the same ordered selection with those counts
         int *cv = a.v_cnt ? a.v_cnt : b.counts, *cs = a.s_cnt ? a.s_cnt : b.counts + a.n_heads;
-        e = run_topp_counts(b.vert, a.n_heads, a.n, false, nullptr, a.p_vertical, a.n_vertical, cv,
-                            b.topp_scratch, st);
-        if (e == cudaSuccess)
-            e = run_topp_counts(b.slash, a.n_heads, a.n, true, b.diag0, a.p_slash, a.n_slash, cs,
-                                b.topp_scratch, st);
+        e = run_topp_counts2(b.vert, a.n_heads, false, nullptr, a.p_vertical, a.n_vertical, cv, b.slash, a.n_heads,
+                             true, b.diag0, a.p_slash, a.n_slash, cs, a.n, b.topp_scratch, st);
         if (e != cudaSuccess) return e;
         kv = cv;
         ks = cs;
