@@ -422,7 +422,8 @@ def main():
             raise SystemExit(f"--shard heads needs at most {w.hkv} ranks (one kv-head each)")
         seed = args.seed
         pats_all = synth.mixed_head_patterns(w, seed) if w.pattern == "mixed" else [w.pattern] * w.hq
-        parts = shard.partition_heads(pats_all, w.hkv, world)
+        parts = shard.partition_heads(pats_all, w.hkv, world, w.n, n_vertical=w.n_vertical, n_slash=w.n_slash,
+                                      topk=w.topk, n_sink=w.n_sink, window=w.window, n_last=w.last_q)
         mine = parts[rank]
         grp = w.hq // w.hkv
         kvs = sorted({h // grp for h in mine})

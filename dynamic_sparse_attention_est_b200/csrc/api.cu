@@ -828,32 +828,80 @@ const char *minf_last_error(void) { return g_last_error.c_str(); }
 // that loads the library holds until the process exits.  Requests whose
 // scratch would exceed it are rejected with MINF_ERR_WORKSPACE.
 //
-// The array's device address is looked up once per device, by the first call
-// made on that device (with that device current); make that first call before
-// any stream capture.  Every call shares the array: calls whose work overlaps
-// on the GPU (different streams, or different host threads, with no ordering
-// between them) race on it.  The status block at its start is cleared by each
-// call; device-side timeouts are therefore not reported by this variant.
+// The array's device address is looked up by the first call made on a device
+// in a given CUDA context (with that device current) and kept for that
+// context; a call from another context, or after the context was reset, looks
+// it up again, since the module and its array may then sit elsewhere.  Make
+// the first call before any stream capture.  Every call shares the array:
+// calls whose work overlaps on the GPU (different streams, or different host
+// threads, with no ordering between them) race on it.  The status block at
+// its start is cleared by each call and read back (and cleared) by
+// minf_vs_estimate_noalloc_status.
 namespace minf {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[64] = {nullptr};
+// Context identity through driver entry points (the library links no libcuda).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
 
+// Id of the context current on this thread, or 0 if it cannot be told.
+unsigned long long current_ctx_id() {
+    std::call_once(g_ctx_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &qres) ==
+                cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+    });
+    if (!g_ctx_current || !g_ctx_id) return 0;
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    return g_ctx_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+struct NoAllocSlot {
+    unsigned long long ctx;  // context the address belongs to (0: none cached)
+    void *ptr;
+};
+std::mutex g_noalloc_mutex;
+NoAllocSlot g_noalloc[64] = {};
+
+// Device address of the built-in array on device `dev`, which must be current.
 int noalloc_scratch(int dev, void **out) {
     std::lock_guard<std::mutex> lk(g_noalloc_mutex);
     if (dev < 0 || dev >= 64) return fail(MINF_ERR_UNSUPPORTED, "device %d out of range", dev);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_ctx_id();
+    NoAllocSlot &slot = g_noalloc[dev];
+    if (ctx == 0 || slot.ctx != ctx || !slot.ptr) {
         void *p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-        g_noalloc_ptr[dev] = p;
+        slot.ctx = ctx;  // 0 (context unknown) caches nothing: the next call looks it up again
+        slot.ptr = p;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return MINF_OK;
+}
+
+// Makes `device` current and returns the built-in array on it.
+int noalloc_on_device(int device, void **out) {
+    int count = 0;
+    cudaError_t e = cudaGetDeviceCount(&count);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+    if (device < 0 || device >= count) return fail(MINF_ERR_INVALID, "device %d out of range", device);
+    e = cudaSetDevice(device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    return noalloc_scratch(device, out);
 }
 
 }  // namespace
@@ -886,4 +934,19 @@ extern "C" int minf_vs_estimate_noalloc(const minf_bf16 *q, const minf_bf16 *k, 
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
     return do_vs_estimate(c, q, k, last_q, n_vertical, n_slash, scale, v_idx, s_idx, ws,
                           static_cast<char *>(ws) + MINF_STATUS_BYTES, st);
+}
+
+extern "C" int minf_vs_estimate_noalloc_status(int device, minf_stream_t stream) {
+    void *ws = nullptr;
+    int rc = noalloc_on_device(device, &ws);
+    if (rc) return rc;
+    return minf_status(ws, stream);  // waits for `stream`, reads and clears the status word
+}
+
+extern "C" int minf_vs_estimate_noalloc_check_timeout(int device, uint64_t limit_ns, minf_stream_t stream) {
+    void *ws = nullptr;
+    int rc = noalloc_on_device(device, &ws);
+    if (rc) return rc;
+    const cudaError_t e = run_wait_timeout_check(ws, limit_ns, (cudaStream_t)stream);
+    return e == cudaSuccess ? MINF_OK : cuda_fail(e, "wait check launch");
 }

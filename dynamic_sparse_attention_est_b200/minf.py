@@ -54,6 +54,8 @@ _SIGS = {
     "minf_dense_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_mixed_layer": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "minf_vs_estimate_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P]),
+    "minf_vs_estimate_noalloc_status": (_I, [_I, _P]),
+    "minf_vs_estimate_noalloc_check_timeout": (_I, [_I, _U64, _P]),
     "minf_status": (_I, [_P, _P]),
     "minf_stats": (_I, [_P, _P, ctypes.POINTER(_U64), ctypes.POINTER(_U64)]),
     "minf_set_wait_limit_ns": (None, [_U64]),
@@ -194,6 +196,18 @@ def minf_vs_estimate_noalloc(q, k, last_q: int = 64, n_vertical: int = 1000, n_s
                                           _scale(scale), ids, nh, _ptr(v_idx), _ptr(s_idx), _stream(q.device)),
            "minf_vs_estimate_noalloc")
     return v_idx, s_idx
+
+
+def minf_vs_estimate_noalloc_status(device=None) -> int:
+    """Status code of the last allocation-free estimate on `device` (read and cleared)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(lib().minf_vs_estimate_noalloc_status(dev.index or 0, _stream(dev)))
+
+
+def minf_vs_estimate_noalloc_check_timeout(limit_ns: int, device=None) -> None:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check(lib().minf_vs_estimate_noalloc_check_timeout(dev.index or 0, int(limit_ns), _stream(dev)),
+           "minf_vs_estimate_noalloc_check_timeout")
 
 
 def _vs_attention(fn_name, q, k, v, v_idx, s_idx, scale, head_ids, out, want_lse, ws):

@@ -9,14 +9,72 @@ is the max-over-ranks reduction of the measured time.
 """
 from __future__ import annotations
 
+import functools
+import math
 from typing import Dict, List, Sequence
 
+import numpy as np
 import torch
 
-# Relative cost of one q-head by pattern: the share of the causal key tiles its
-# mask makes the kernel compute, measured on the 1M-token synthetic layer
-# (Vertical-Slash ~0.5, Block-Sparse 100/16384 blocks, A-shape 4224/1M keys).
-PATTERN_COST = {"dense": 1.0, "vs": 0.5, "block": 0.0125, "ashape": 0.005, "trishape": 0.006}
+# Relative cost of one q-head by pattern: the 128x128 tiles the attention
+# kernel computes for it at n tokens, from the kernel's own tile plan (dense,
+# A-shape, Tri-shape exactly; Block-Sparse and Vertical-Slash from their
+# budgets under a model of the index sets, see `head_tiles`), as a share of the
+# dense causal head.  A Vertical-Slash head at 32K tokens costs a dense head
+# (its 6,096 slash ranges cover every causal tile); at 1M about half of one.
+DEFAULT_PARAMS = dict(n_vertical=1000, n_slash=6096, topk=100, n_sink=128, window=4096, n_last=64)
+
+
+@functools.lru_cache(maxsize=256)
+def head_tiles(pattern: str, n: int, n_vertical: int = 1000, n_slash: int = 6096, topk: int = 100,
+               n_sink: int = 128, window: int = 4096, n_last: int = 64) -> float:
+    """Predicted 128x128 tiles (two 64-key halves each) computed for one q-head.
+
+    Per 128-row query tile t (rows r0 = 128 t ...):
+      dense          the causal halves, min(2t + 2, n / 64);
+      ashape         the sink halves plus the window halves (or the causal ones
+                     where they meet), as the kernel's tile plan walks them;
+      trishape       the same, with tiles holding the last n_last rows dense;
+      block          the union of the two query blocks' lists of min(topk, b + 1)
+                     blocks, their overlap taken as that of independent draws
+                     from the causal prefix;
+      vs             slash offsets spread evenly over [0, n): each reaches a
+                     128-key range, so a key is covered with probability
+                     1 - exp(-128 n_slash / n); the verticals fill the uncovered
+                     rest, 64 per half.
+    """
+    nb64 = n // 64
+    t = np.arange((n + 127) // 128, dtype=np.float64)
+    r0 = 128.0 * t
+    hi = np.minimum(2.0 * t + 1, nb64 - 1)
+    causal = hi + 1
+    if pattern == "dense":
+        halves = causal
+    elif pattern in ("ashape", "trishape"):
+        sink_h = min(-(-n_sink // 64), nb64)
+        w_lo = np.floor(np.maximum(0.0, r0 - window + 1) / 64)
+        split = w_lo > sink_h
+        if pattern == "trishape":
+            split &= np.minimum(r0 + 127, n - 1) < n - n_last
+        halves = np.where(split, sink_h + (hi - w_lo + 1), causal)
+    elif pattern == "block":
+        b0, b1 = 2.0 * t, 2.0 * t + 1
+        k0 = np.minimum(topk, b0 + 1)
+        k1 = np.where(b1 < nb64, np.minimum(topk, b1 + 1), 0.0)
+        halves = np.minimum(causal, k0 + k1 - k0 * k1 / (b1 + 1))
+    elif pattern == "vs":
+        keys = np.minimum(r0 + 128, n)
+        cov = 1.0 - math.exp(-128.0 * min(n_slash, n) / n)
+        halves = np.minimum(causal, keys * cov / 64 + np.minimum(n_vertical, keys) * (1 - cov) / 64 + 1)
+    else:
+        raise ValueError(pattern)
+    return float(np.ceil(halves / 2).sum())
+
+
+def pattern_cost(pattern: str, n: int, **params) -> float:
+    """Cost of one q-head of `pattern` at n tokens, relative to a dense causal head."""
+    p = {**DEFAULT_PARAMS, **params}
+    return head_tiles(pattern, n, **p) / head_tiles("dense", n)
 
 
 def rank_seed(seed: int, rank: int) -> int:
@@ -24,18 +82,20 @@ def rank_seed(seed: int, rank: int) -> int:
     return seed + 1009 * rank
 
 
-def partition_heads(head_patterns: Sequence[str], hkv: int, world: int) -> List[List[int]]:
+def partition_heads(head_patterns: Sequence[str], hkv: int, world: int, n: int = 1 << 20,
+                    **params) -> List[List[int]]:
     """Longest-processing-time assignment of whole GQA groups to ranks.
 
     A group (one kv-head and its q-heads) stays on one rank so that its K and V
-    are read by one GPU only.  Returns, per rank, the ascending q-head ids.
+    are read by one GPU only; each head weighs `pattern_cost` at n tokens with
+    the layer's pattern parameters.  Returns, per rank, the ascending q-head ids.
     """
     hq = len(head_patterns)
     grp = hq // hkv
     costs = []
     for g in range(hkv):
         heads = list(range(g * grp, (g + 1) * grp))
-        costs.append((sum(PATTERN_COST[head_patterns[h]] for h in heads), g, heads))
+        costs.append((sum(pattern_cost(head_patterns[h], n, **params) for h in heads), g, heads))
     costs.sort(key=lambda c: (-c[0], c[1]))
     load = [0.0] * world
     out: List[List[int]] = [[] for _ in range(world)]
@@ -57,8 +117,9 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def shard_summary(parts: List[List[int]], head_patterns: Sequence[str]) -> Dict[int, float]:
-    return {r: sum(PATTERN_COST[head_patterns[h]] for h in p) for r, p in enumerate(parts)}
+def shard_summary(parts: List[List[int]], head_patterns: Sequence[str], n: int = 1 << 20,
+                  **params) -> Dict[int, float]:
+    return {r: sum(pattern_cost(head_patterns[h], n, **params) for h in p) for r, p in enumerate(parts)}
 
 
 def gather_heads(local: torch.Tensor, parts: List[List[int]], hq: int) -> torch.Tensor:

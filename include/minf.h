@@ -287,15 +287,36 @@ int minf_selftest_exp2(const float *x, float *y_poly, float *y_hw, int n, minf_s
  * the library that every GPU loading the library keeps until the process
  * exits.  Calls needing more scratch than that (as sized by
  * minf_workspace_bytes(MINF_OP_VS_ESTIMATE, ...)) return MINF_ERR_WORKSPACE.
- * The first call on a device looks up the array's address on that device:
- * make it before any stream capture.  All calls share the array, so calls
- * that may overlap on the GPU race; order them on one stream.  Device-side
- * timeouts are not reported by this variant.
+ * The first call on a device, in a given CUDA context, looks up the array's
+ * address there (a later context, or a reset one, looks it up again): make
+ * that first call before any stream capture.  All calls share the array, so
+ * calls that may overlap on the GPU race; order them on one stream.  Each call
+ * clears the status block at the start of the array; a device-side timeout of
+ * the call is read back with minf_vs_estimate_noalloc_status.
  */
 int minf_vs_estimate_noalloc(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
                              int last_q, int n_vertical, int n_slash, float scale,
                              const int32_t *head_ids, int n_heads, int32_t *v_idx, int32_t *s_idx,
                              minf_stream_t stream);
+
+/*
+ * Status of the last minf_vs_estimate_noalloc on `device` (no counterpart in
+ * the method's sources): makes `device` current, waits for `stream`, returns
+ * MINF_OK or the device-side error the call recorded in the built-in array's
+ * status block (MINF_ERR_TIMEOUT: a bounded wait ran out and the returned
+ * indices are not valid; minf_last_error() names where), and clears it.  Like
+ * minf_status for the workspace calls.  MINF_ERR_INVALID for a device ordinal
+ * out of range.
+ */
+int minf_vs_estimate_noalloc_status(int device, minf_stream_t stream);
+
+/*
+ * Self-test of that read-back (no counterpart in the method's sources): on
+ * `device`, launches one bounded wait that nothing satisfies, which gives up
+ * after limit_ns and records MINF_ERR_TIMEOUT in the built-in array's status
+ * block, as a timed-out estimate would.  Asynchronous on `stream`.
+ */
+int minf_vs_estimate_noalloc_check_timeout(int device, uint64_t limit_ns, minf_stream_t stream);
 
 /* Library version string and the message of the last host-side error. */
 const char *minf_version(void);

@@ -5,8 +5,11 @@
   within 1e-2 absolute (fp32 accumulation, ex2.approx).
 * Index sets: with t the oracle's k-th best score, every item scoring above
   t + band is in the GPU set, every item below t - band is not, and the set
-  holds exactly k items; band = 1e-3 |t| + 1e-6 (the relative 1e-3 tie band,
-  with an absolute floor for scores that sit near zero).
+  holds exactly k items.  band = 1e-3 |t| (the relative tie band) for the
+  Vertical-Slash column and diagonal sums, which are positive sums of softmax
+  weights.  Block-Sparse pooled scores are raw dot products that can sit at
+  or near zero, where a relative band vanishes; their band adds twice the
+  worst-case fp32 error of the GPU's pooled score (`bs_score_error`).
 """
 from __future__ import annotations
 
@@ -17,7 +20,47 @@ MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 1e-2
 REL_BAND = 1e-3
-ABS_BAND = 1e-6
+U32 = 2.0 ** -24  # unit roundoff of fp32
+
+
+def _gamma(m):
+    """Higham's gamma_m = m u / (1 - m u): the relative error bound of m sequential fp32 roundings."""
+    return m * U32 / (1.0 - m * U32)
+
+
+# Worst-case error of one GPU pooled score s^_ij against the exact dot product of
+# the exact block means, in units of sum_d a_i,d * b_j,d with a, b the block means
+# of |q| and |k|.  The GPU sums the 64 bf16 rows of a block in fp32, one rounding
+# per add (63; the first add is exact) and scales by 1/64 (exact), so each pooled
+# value is off by at most gamma_63 a (or b); it then accumulates the 128 products
+# with one fp32 FMA each, off by at most gamma_128 sum |p^q||p^k|.  With
+# |p| <= a and |p^| <= (1 + gamma_63) a:
+#   |s^ - s| <= [gamma_128 (1 + gamma_63)^2 + 2 gamma_63 + gamma_63^2] sum_d a_d b_d.
+BS_ERR_COEF = _gamma(128) * (1 + _gamma(63)) ** 2 + 2 * _gamma(63) + _gamma(63) ** 2
+
+
+def bs_score_error(q, k, block=64):
+    """Per (q-head, query block i): twice the largest worst-case fp32 error of the
+    GPU's pooled scores s_ij over the candidates j < i (zero for i = 0).
+
+    With that error at most E on every candidate of a row, an item whose exact
+    score exceeds the k-th best exact score t by more than 2E outranks, on the GPU,
+    every item that does not score above t exactly -- at most k - 1 others -- so it
+    must be selected; symmetrically below t - 2E.  q: [hq][n][128], k: [hkv][n][128]
+    (bf16 tensors or arrays; GQA groups contiguous)."""
+    qa = np.abs(to_np(q))
+    ka = np.abs(to_np(k))
+    hq, n, d = qa.shape
+    hkv = ka.shape[0]
+    nb = n // block
+    aq = qa.reshape(hq, nb, block, d).mean(axis=2)
+    ak = ka.reshape(hkv, nb, block, d).mean(axis=2)
+    out = np.zeros((hq, nb))
+    below = np.tril(np.ones((nb, nb), bool), -1)
+    for h in range(hq):
+        m = aq[h] @ ak[h // (hq // hkv)].T
+        out[h] = 2.0 * BS_ERR_COEF * np.where(below, m, 0.0).max(axis=1)
+    return out
 
 
 def to_np(t):
@@ -48,8 +91,9 @@ def check_attention(gpu_out, gpu_lse, ref_out, ref_lse, what=""):
     return float(err.max()), float(err.mean())
 
 
-def check_topk_band(gpu_idx, scores, k, what=""):
-    """gpu_idx: 1-D indices (-1 padded); scores: oracle fp64 scores of every candidate."""
+def check_topk_band(gpu_idx, scores, k, what="", abs_band=0.0):
+    """gpu_idx: 1-D indices (-1 padded); scores: oracle fp64 scores of every candidate.
+    abs_band: added to the relative band (Block-Sparse rows: `bs_score_error`)."""
     scores = np.asarray(scores, np.float64)
     kk = min(k, len(scores))
     got = [int(x) for x in np.asarray(gpu_idx).ravel() if x >= 0]
@@ -60,7 +104,7 @@ def check_topk_band(gpu_idx, scores, k, what=""):
         return 0
     order = np.sort(scores)[::-1]
     t = order[kk - 1]
-    band = REL_BAND * abs(t) + ABS_BAND if np.isfinite(t) else 0.0
+    band = REL_BAND * abs(t) + abs_band if np.isfinite(t) else 0.0
     gs = set(got)
     must = np.nonzero(scores > t + band)[0]
     never = np.nonzero(scores < t - band)[0]

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from dynamic_sparse_attention_est_b200 import minf, synth
-from parity import check_attention, check_topk_band
+from parity import bs_score_error, check_attention, check_topk_band
 
 pytestmark = pytest.mark.gpu
 
@@ -100,9 +100,10 @@ def test_block_128k_layer(orc):
         qh, kh, vh = head_inputs(x, h, grp)
         obi, obc, _, _, sc = orc.block_estimate(qh, kh, 64, w.topk, return_scores=True)
         gbi, gbc = bi[h].cpu().numpy(), bc[h].cpu().numpy()
+        eb = bs_score_error(qh, kh)[0]
         for i in list(range(0, nb, 37)) + [nb - 1]:
             assert gbc[i] == min(w.topk, i + 1) and gbi[i, gbc[i] - 1] == i
-            check_topk_band(gbi[i, :gbc[i] - 1], sc[0, i, :i], w.topk - 1, f"block row {h}/{i}")
+            check_topk_band(gbi[i, :gbc[i] - 1], sc[0, i, :i], w.topk - 1, f"block row {h}/{i}", abs_band=eb[i])
         ref, rl = orc.block_attention(qh, kh, vh, SCALE, 64, gbi[None], gbc[None], rows=rows)
         check_attention(out[h, rows], lse[h, rows], ref[0], rl[0], f"block 128K head {h}")
         o2, l2 = minf.minf_block_attention(q, k, v, torch.from_numpy(obi).cuda(), torch.from_numpy(obc).cuda(),

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from dynamic_sparse_attention_est_b200 import minf, synth
-from parity import check_attention, check_topk_band, check_topp, to_np
+from parity import bs_score_error, check_attention, check_topk_band, check_topp, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -74,12 +74,13 @@ def test_block_estimate_band(orc, n, hq, hkv, topk):
     gi, gc = minf.minf_block_estimate(*cuda(q, k), topk=topk)
     gi, gc = gi.cpu().numpy(), gc.cpu().numpy()
     nb = n // 64
+    eb = bs_score_error(q, k)
     for hp in range(hq):
         for i in range(nb):
             row = gi[hp, i, :gc[hp, i]]
             assert gc[hp, i] == min(topk, i + 1)
             assert row[-1] == i, "diagonal block forced"
-            check_topk_band(row[:-1], sc[hp, i, :i], topk - 1, f"block row {hp}/{i}")
+            check_topk_band(row[:-1], sc[hp, i, :i], topk - 1, f"block row {hp}/{i}", abs_band=eb[hp, i])
             assert np.all(gi[hp, i, gc[hp, i]:] == -1)
 
 

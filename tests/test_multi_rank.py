@@ -57,19 +57,47 @@ def test_two_gloo_ranks_assemble_the_layer(tmp_path):
     assert overlap == 0 and total == 8
 
 
-def test_partition_is_balanced_and_keeps_groups_whole():
+@pytest.mark.parametrize("n", [32768, 1 << 20])
+def test_partition_is_balanced_and_keeps_groups_whole(n):
     w = synth.WORKLOADS["mixed-gqa-1m"]
     pats = synth.mixed_head_patterns(w, seed=0)
+    cost = {p: shard.pattern_cost(p, n) for p in set(pats)}
     for world in (1, 2, 4, 8):
-        parts = shard.partition_heads(pats, 8, world)
+        parts = shard.partition_heads(pats, 8, world, n)
         flat = sorted(h for p in parts for h in p)
         assert flat == list(range(32))
         for p in parts:
             assert all(((h // 4) * 4 + i) in p for h in p for i in range(4))  # whole groups
-        loads = shard.shard_summary(parts, pats)
-        if world <= 8:
-            heaviest_group = max(sum(shard.PATTERN_COST[pats[g * 4 + i]] for i in range(4)) for g in range(8))
-            assert max(loads.values()) - min(loads.values()) <= heaviest_group + 1e-9
+        loads = shard.shard_summary(parts, pats, n)
+        heaviest_group = max(sum(cost[pats[g * 4 + i]] for i in range(4)) for g in range(8))
+        assert max(loads.values()) - min(loads.values()) <= heaviest_group + 1e-9
+
+
+def test_pattern_costs_follow_the_tile_plan():
+    """Closed forms against hand counts of the kernel's tile plan."""
+    # dense causal at 256 tokens: query tiles 0 and 1 compute 1 and 2 tiles
+    assert shard.head_tiles("dense", 256) == 3
+    # A-shape whose window covers everything is dense
+    assert shard.head_tiles("ashape", 4096, window=4096) == shard.head_tiles("dense", 4096)
+    # Tri-shape with every row in the dense tail is dense; with none it is A-shape
+    assert shard.head_tiles("trishape", 8192, n_last=8192) == shard.head_tiles("dense", 8192)
+    assert shard.head_tiles("trishape", 8192, n_last=0) == shard.head_tiles("ashape", 8192)
+    # A-shape at 128K, counted tile by tile: 2 sink halves, then the window's halves
+    # from the one holding key r0 - 4095 up to the diagonal half (or every causal
+    # half while the window still reaches the sinks)
+    n, tiles = 131072, 0
+    for t in range(n // 128):
+        r0, hi = 128 * t, 2 * t + 1
+        w_lo = max(0, r0 - 4095) // 64
+        halves = (2 + hi - w_lo + 1) if w_lo > 2 else hi + 1
+        tiles += (halves + 1) // 2  # a tile is two halves
+    assert shard.head_tiles("ashape", n) == tiles
+    # Block-Sparse with every block selected is dense
+    assert shard.head_tiles("block", 4096, topk=64) == shard.head_tiles("dense", 4096)
+    # Vertical-Slash: at 32K the slash ranges cover the causal tiles; at 1M about half
+    assert shard.pattern_cost("vs", 32768) > 0.99
+    assert 0.4 < shard.pattern_cost("vs", 1 << 20) < 0.7
+    assert shard.pattern_cost("block", 1 << 20) < shard.pattern_cost("block", 32768)
 
 
 def test_rank_seeds_differ():
