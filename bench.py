@@ -8,7 +8,8 @@ A step is one pass of the whole path over one layer of synthetic input:
   ashape-gqa-128k  minf_ashape_attention (128K tokens)
   trishape-gqa-128k minf_trishape_attention (A-shape + dense last 64 rows, 128K tokens)
   mixed-gqa-1m     minf_mixed_layer, per-head patterns drawn from the seed (1M tokens)
-The default is vs-gqa-32k.  Inputs stay resident in HBM and are larger than L2,
+The default is mixed-gqa-1m, the layer the 1M-token targets are stated on.
+Inputs stay resident in HBM and are larger than L2,
 so no flush is needed between steps.  The line also carries the roofline of the
 attention kernel (computed-tile FLOPs / its CUDA-event time), the same metric
 end to end from pinned host buffers, the dense causal kernel on the same
@@ -47,9 +48,9 @@ TILE_FLOPS = 4 * 128 * 128 * 128  # QK^T and PV of one 128x128 tile, d = 128
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 20; 5 at 1M tokens)")
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="vs-gqa-32k")
+    ap.add_argument("--workload", default="mixed-gqa-1m")
     ap.add_argument("--impl", default="minf", choices=["minf", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--shard", default="layers", choices=["layers", "heads"],
@@ -59,10 +60,20 @@ def parse():
                     help="Vertical-Slash top-p budgets (p for verticals and slashes; the budgets become caps)")
     ap.add_argument("--vs-mode", default="exact", choices=["exact", "tiles"],
                     help="Vertical-Slash key set: token-exact, or every computed slash range attended whole")
+    ap.add_argument("--vs-diag-ratio", type=float, default=None,
+                    help="Vertical-Slash routing: slash groups of m offsets over H half-tiles run on the CUDA "
+                         "cores when m < ratio * H (0: tensor cores only; default: the library's)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-kernel comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work to sample")
-    return ap.parse_args()
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle attention rows to sample")
+    ap.add_argument("--cpu-mode", default="auto", choices=["auto", "full", "sample"],
+                    help="CPU baseline: the whole layer (auto up to 32K tokens) or a bounded sample, projected")
+    a = ap.parse_args()
+    if a.steps is None:
+        from dynamic_sparse_attention_est_b200 import synth
+
+        a.steps = 5 if synth.WORKLOADS[a.workload].n > 131072 else 20
+    return a
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
@@ -104,6 +115,55 @@ def pick_bf16_peak(peaks, elapsed_ms, clk):
         sustained = elapsed_ms >= 1000.0 or "sw_power_cap" in (clk.get("reasons") or [])
     key = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     return peaks.get(key), key
+
+
+# Peak fp32 FMA rate of the CUDA cores, from the unit counts: 148 SMs x 4
+# sub-partitions x 32 FMA lanes, 2 FLOP per FMA, at the SM clock.
+def alu_peak_tflops(sm_mhz: float) -> float:
+    return 148 * 4 * 32 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def kernel_rooflines(kernels, detail, peaks, src, peak, peak_key, elapsed, clk, traffic_key):
+    """(roofline of the kernel with the largest share of the timed region, roofline of
+    the attention tile kernel with the largest share) from the live per-kernel times.
+
+    attn_kernel<P>: computed-tile FLOPs (4 x 128^3 per 128x128 tile, tiles of that
+    kernel from the counters) per launch over its average launch time, against the
+    bf16 tensor peak.  vs_diag_kernel: useful FLOPs (2 x 128 multiply-adds per
+    (query, key) pair, QK^T and PV) per launch over its launch time, against the
+    fp32 FMA peak of the CUDA cores at the maximum SM clock."""
+    pat_key = {"attn_kernel<DENSE>": "tiles_dense", "attn_kernel<VS>": "tiles_vs",
+               "attn_kernel<BLOCK>": "tiles_block", "attn_kernel<ASHAPE>": "tiles_ashape"}
+
+    def one(name):
+        k = kernels[name]
+        sec = k["ms_per_launch"] * 1e-3
+        if name in pat_key:
+            flops = detail.get(pat_key[name], 0) * TILE_FLOPS
+            ach = flops / sec / 1e12
+            return {"kernel": name, "bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(ach / peak, 4), "flops_per_launch": flops,
+                    "traffic": attention_traffic(traffic_key) if name == "attn_kernel<VS>" else None,
+                    "ms_per_launch": k["ms_per_launch"],
+                    "peak_source": f"{src} {peak_key} (timed region {elapsed:.0f} ms, median SM clock "
+                                   f"{clk.get('sm_mhz')} MHz)"}
+        if name == "vs_diag_kernel":
+            flops = 4 * 128 * detail.get("diag_pairs", 0)
+            ach = flops / sec / 1e12
+            pk = alu_peak_tflops(peaks.get("sm_max_mhz") or 1965.0)
+            return {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(pk, 1),
+                    "unit": "TFLOP/s", "frac": round(ach / pk, 4), "flops_per_launch": flops, "traffic": None,
+                    "ms_per_launch": k["ms_per_launch"],
+                    "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x max SM clock"}
+        return {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
+                "traffic": None, "ms_per_launch": k["ms_per_launch"]}
+
+    if not kernels:
+        return None, None
+    top = max(kernels, key=lambda n: kernels[n]["ms_total"])
+    attn = [n for n in kernels if n in pat_key]
+    top_attn = max(attn, key=lambda n: kernels[n]["ms_total"]) if attn else None
+    return one(top), (one(top_attn) if top_attn else None)
 
 
 def measured_peaks():
@@ -305,61 +365,117 @@ def estimate_bytes(w) -> float:
     return 0.0
 
 
-def cpu_sample(w, x, orc, budget_s, seed, vs_mode="exact"):
-    """Times the fp64 oracle on a bounded sample of the workload and scales it to one layer."""
+def _time_rows(w, pattern, orc, q1, k1, v1, scale, idx, budget_s, vs_mode):
+    """Seconds per attention row of one head, over rows spread across the sequence,
+    grown until about half of `budget_s` is spent (the oracle spreads rows over
+    its threads, so a layer's rows scale linearly)."""
     import numpy as np
-    import torch
 
-    scale = 1.0 / math.sqrt(128)
-    hq, hkv, n = w.hq, w.hkv, w.n
-    g = hq // hkv
-    # one q-head (and its kv-head) as float32 host arrays
-    q1 = x["q"][0:1].float().cpu().numpy()
-    k1 = x["k"][0:1].float().cpu().numpy()
-    v1 = x["v"][0:1].float().cpu().numpy()
-    est_s = 0.0
-    detail = []
-    t0 = time.perf_counter()
-    if w.pattern in ("vs", "mixed"):
-        vi, si = orc.vs_estimate(q1, k1, w.last_q, w.n_vertical, w.n_slash, scale)
-        est_s = time.perf_counter() - t0
-        detail.append(f"VS estimate of 1 head ({est_s:.2f} s) x {hq}")
-    elif w.pattern == "block":
-        if n // 64 <= 4096:
-            bi, bc = orc.block_estimate(q1, k1, 64, w.topk)
-            est_s = time.perf_counter() - t0
-            detail.append(f"block estimate of 1 head ({est_s:.2f} s) x {hq}")
-    # attention rows: spread over the sequence, grown until the budget is used
-    rows_per_s = None
-    nrows = 64
-    spent = 0.0
+    n = w.n
+    nrows, spent = 64, 0.0
     while True:
         rows = np.linspace(0, n - 1, nrows).astype(np.int32)
         t1 = time.perf_counter()
-        if w.pattern == "vs" and vs_mode == "tiles":
-            orc.vs_tiles_attention(q1, k1, v1, scale, vi, si, 128, rows=rows)
-        elif w.pattern in ("vs", "mixed"):
-            orc.vs_attention(q1, k1, v1, scale, vi, si, rows=rows)
-        elif w.pattern == "block":
-            if n // 64 > 4096:
-                bi = np.tile(np.arange(w.topk, dtype=np.int32), (1, n // 64, 1))
-                bc = np.full((1, n // 64), w.topk, np.int32)
-            orc.block_attention(q1, k1, v1, scale, 64, bi, bc, rows=rows)
-        elif w.pattern == "trishape":
+        if pattern == "vs" and vs_mode == "tiles":
+            orc.vs_tiles_attention(q1, k1, v1, scale, idx[0], idx[1], 128, rows=rows)
+        elif pattern == "vs":
+            orc.vs_attention(q1, k1, v1, scale, idx[0], idx[1], rows=rows)
+        elif pattern == "block":
+            orc.block_attention(q1, k1, v1, scale, 64, idx[0], idx[1], rows=rows)
+        elif pattern == "trishape":
             orc.trishape_attention(q1, k1, v1, scale, w.n_sink, w.window, w.last_q, rows=rows)
-        else:
+        elif pattern == "ashape":
             orc.ashape_attention(q1, k1, v1, scale, w.n_sink, w.window, rows=rows)
+        else:
+            orc.dense_attention(q1, k1, v1, scale, rows=rows)
         dt = time.perf_counter() - t1
         spent += dt
-        rows_per_s = nrows / dt
         if spent > budget_s * 0.5 or nrows >= n:
-            break
+            return dt / nrows, nrows
         nrows = min(n, int(nrows * max(2.0, (budget_s * 0.5) / max(dt, 1e-3))))
-    attn_layer_s = hq * n / rows_per_s
-    layer_s = est_s * hq + attn_layer_s
-    detail.append(f"attention of {nrows} rows spread over the sequence of 1 head, scaled to {hq} x {n} rows")
-    return {"value": layer_s * 1000.0, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
-            "sample": "; ".join(detail)}
+
+
+def cpu_estimates(w, pattern, orc, q1, k1, scale):
+    """One head's index estimate for `pattern`: (seconds, indices for the row timing, note).
+
+    Block-Sparse estimates beyond 4,096 blocks (their pooled-score triangle grows
+    with the square of the block count) are timed on the first 2,048 blocks and
+    scaled by (blocks / 2,048)^2; the row timing then uses the first topk blocks
+    of each row, which has the same number of keys as any top-k list."""
+    import numpy as np
+
+    t0 = time.perf_counter()
+    if pattern == "vs":
+        vi, si = orc.vs_estimate(q1, k1, w.last_q, w.n_vertical, w.n_slash, scale)
+        return time.perf_counter() - t0, (vi, si), "estimate of 1 head timed"
+    if pattern == "block":
+        nb = w.n // 64
+        if nb <= 4096:
+            bi, bc = orc.block_estimate(q1, k1, 64, w.topk)
+            return time.perf_counter() - t0, (bi, bc), "estimate of 1 head timed"
+        m = 2048 * 64
+        orc.block_estimate(q1[:, :m], k1[:, :m], 64, w.topk)
+        dt = (time.perf_counter() - t0) * (nb / 2048) ** 2
+        bi = np.tile(np.arange(w.topk, dtype=np.int32), (1, nb, 1))
+        bc = np.full((1, nb), w.topk, np.int32)
+        return dt, (bi, bc), f"estimate of 1 head timed on 2,048 blocks, scaled by ({nb}/2048)^2"
+    return 0.0, None, ""
+
+
+def cpu_sample(w, x, orc, budget_s, vs_mode="exact", pats=None, full=False, cache=None):
+    """The fp64 oracle on the host cores, as the CPU baseline of one layer.
+
+    full: every head's estimate and every row's attention are run (feasible up
+    to 32K tokens); x then holds the whole layer.  Otherwise x holds one q-head
+    and its kv-head, and the layer is projected from a bounded sample, per
+    pattern present: one head's estimate (the oracle runs one head per thread,
+    so the layer's estimates of c heads take ceil(c / threads) of it) plus
+    attention rows spread over the sequence, scaled to c x n rows.  `cache`
+    keeps the estimates between calls (the reference arm re-times rows only).
+    """
+    import numpy as np
+
+    scale = 1.0 / math.sqrt(128)
+    threads = orc.threads()
+    t_start = time.perf_counter()
+    if full:
+        q, k, v = (x[key].float().cpu().numpy() for key in ("q", "k", "v"))
+        t0 = time.perf_counter()
+        if w.pattern == "vs":
+            vi, si = orc.vs_estimate(q, k, w.last_q, w.n_vertical, w.n_slash, scale)
+            est = time.perf_counter() - t0
+            if vs_mode == "tiles":
+                orc.vs_tiles_attention(q, k, v, scale, vi, si, 128)
+            else:
+                orc.vs_attention(q, k, v, scale, vi, si)
+        elif w.pattern == "block":
+            bi, bc = orc.block_estimate(q, k, 64, w.topk)
+            est = time.perf_counter() - t0
+            orc.block_attention(q, k, v, scale, 64, bi, bc)
+        else:
+            raise ValueError("full CPU timing covers the Vertical-Slash and Block-Sparse layers")
+        total = time.perf_counter() - t0
+        return {"value": total * 1000.0, "unit": UNIT, "cores": threads, "kind": "oracle", "projected": False,
+                "sample": f"whole layer ({w.hq} heads x {w.n} rows): estimate {est:.2f} s + attention "
+                          f"{total - est:.2f} s, timed", "seconds": round(time.perf_counter() - t_start, 2)}
+    q1, k1, v1 = (x[key][0:1].float().cpu().numpy() for key in ("q", "k", "v"))
+    counts = {}
+    for p in (pats if pats is not None else [w.pattern] * w.hq):
+        counts[p] = counts.get(p, 0) + 1
+    cache = {} if cache is None else cache
+    layer_s, notes = 0.0, []
+    share = budget_s / max(1, len(counts))
+    for p, c in sorted(counts.items()):
+        if p not in cache:
+            cache[p] = cpu_estimates(w, p, orc, q1, k1, scale)
+        est_s, idx, note = cache[p]
+        t_row, nrows = _time_rows(w, p, orc, q1, k1, v1, scale, idx, share, vs_mode)
+        layer_s += math.ceil(c / threads) * est_s + c * w.n * t_row
+        notes.append(f"{p} x{c}: " + (f"{note} ({est_s:.2f} s), x ceil({c}/{threads}); " if note else "") +
+                     f"attention of {nrows} rows of 1 head ({t_row * 1e3:.3f} ms/row), x {c} x {w.n} rows")
+    return {"value": layer_s * 1000.0, "unit": UNIT, "cores": threads, "kind": "oracle", "projected": True,
+            "sample": "projected from a sample -- " + "; ".join(notes),
+            "seconds": round(time.perf_counter() - t_start, 2)}
 
 
 def main():
@@ -379,22 +495,30 @@ def main():
         import torch
 
         orc = oracle.get()
-        # the sample attends with q-head 0 only: draw that head and its kv-head
-        x = synth.generate(w, seed=args.seed, device="cpu", hq=1, hkv=1)
+        pats = synth.mixed_head_patterns(w, args.seed) if w.pattern == "mixed" else None
+        full = args.cpu_mode == "full" or (args.cpu_mode == "auto" and w.n <= 32768 and w.pattern in ("vs", "block"))
+        # a sample needs q-head 0 and its kv-head only; the full layer needs every head
+        x = synth.generate(w, seed=args.seed, device="cpu") if full else \
+            synth.generate(w, seed=args.seed, device="cpu", hq=1, hkv=1)
         per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-        vals = []
+        vals, step_s, cache = [], [], {}
         for i in range(args.warmup + args.steps):
-            r = cpu_sample(w, x, orc, per, args.seed, args.vs_mode)
+            t0 = time.perf_counter()
+            r = cpu_sample(w, x, orc, per, args.vs_mode, pats, full, cache)
             if i >= args.warmup:
                 vals.append(r["value"])
+                step_s.append(time.perf_counter() - t0)
         val = statistics.median(vals)
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
+                "steps": args.steps, "warmup": args.warmup,
+                # wall time of one step of this arm: the timed sample (or the whole layer when not projected)
+                "ms_per_step": round(1000.0 * statistics.mean(step_s), 1), "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "projected": r["projected"],
                 "config": {"workload": w.name, "hq": w.hq, "hkv": w.hkv, "n": w.n,
                            **({"vs_mode": args.vs_mode} if w.pattern == "vs" else {})},
                 "cpu_baseline": {"value": val, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
-                                 "sample": r["sample"]},
+                                 "projected": r["projected"], "sample": r["sample"]},
                 "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return 0
@@ -406,6 +530,8 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.vs_diag_ratio is not None:
+        minf.minf_set_vs_diag_ratio(args.vs_diag_ratio)
     if world > 1:
         from datetime import timedelta
 
@@ -459,8 +585,10 @@ def main():
         torch.cuda.synchronize()
         log(f"warm-up {i}: attention done")
     tiles, pairs = minf.minf_stats(ws)
+    detail = minf.minf_stats_detail(ws)
     if minf.minf_status(ws) != minf.MINF_OK:
         raise RuntimeError("device status not OK after warm-up")
+    minf.minf_profile_read()  # drop anything recorded before the timed region
 
     # ---- timed region: K steps, events around the whole and around each attention call
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -472,6 +600,7 @@ def main():
     clocks.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    minf.minf_profile_enable(True)  # an event pair around each of the library's launches, on its stream
     t_start.record(stream)
     for i in range(args.steps):
         estimate()
@@ -480,6 +609,8 @@ def main():
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    minf.minf_profile_enable(False)
+    kernel_ms = minf.minf_profile_read()
     clk = clocks.stop()
     elapsed = t_start.elapsed_time(t_end)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
@@ -574,19 +705,21 @@ def main():
 
     peaks, src = measured_peaks()
     peak, peak_key = pick_bf16_peak(peaks, elapsed, clk)
-    achieved = tiles * TILE_FLOPS / (attn_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": attention_traffic(w.name if args.vs_mode == "exact" else None),
-                "kernel": "attn_kernel (timed with its plan kernels, CUDA events around the attention call)",
-                "peak_source": f"{src} {peak_key} (timed region {elapsed:.0f} ms, median SM clock {clk.get('sm_mhz')} MHz)"}
+    kernels = {name: {"launches": c, "ms_total": round(ms, 3), "ms_per_launch": round(ms / max(c, 1), 4),
+                      "share": round(ms / elapsed, 4)} for name, (c, ms) in kernel_ms.items()}
+    roofline, tensor_roofline = kernel_rooflines(kernels, detail, peaks, src, peak, peak_key, elapsed, clk,
+                                                 w.name if args.vs_mode == "exact" else None)
 
     log("dense comparison done")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
 
-        xs = {"q": x["q"][:1].cpu(), "k": x["k"][:1].cpu(), "v": x["v"][:1].cpu()}
-        cpu = cpu_sample(w, xs, oracle.get(), args.cpu_budget, seed, args.vs_mode)
+        full = args.cpu_mode == "full" or (args.cpu_mode == "auto" and w.n <= 32768 and w.pattern in ("vs", "block"))
+        pats = synth.mixed_head_patterns(w, seed) if w.pattern == "mixed" else None
+        xs = x if full else {"q": x["q"][:1].cpu(), "k": x["k"][:1].cpu(), "v": x["v"][:1].cpu()}
+        log("CPU baseline: " + ("whole layer" if full else "bounded sample"))
+        cpu = cpu_sample(w, xs, oracle.get(), args.cpu_budget, args.vs_mode, pats, full)
 
     if rank == 0:
         line = {
@@ -605,6 +738,9 @@ def main():
                                        f"output all-gathered (shards {[len(p) for p in parts]})") if sharded
                        else f"one layer per rank x{world}"},
             "roofline": roofline,
+            "tensor_roofline": tensor_roofline,
+            "kernels": kernels,
+            "counters": detail,
             "attention_ms": round(attn_ms, 4),
             "estimate_ms": round(ms_per_step - attn_ms, 4),
             "estimate_roofline": ({"bound": "hbm", "bytes": estimate_bytes(w_run),

@@ -21,6 +21,9 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+// Vertical-Slash routing of sparse slash groups to the CUDA-core pass: a tile
+// half is taken to cost this many offsets of that pass (0: tile kernel only).
+std::atomic<float> g_vs_diag_ratio{2.0f};
 
 int fail(int code, const char *fmt, ...) {
     char buf[512];
@@ -101,6 +104,10 @@ VsPlanBufs carve_vs_plan(Carver &c, int n, int n_heads, int n_vertical, int n_sl
     b.nvert = c.take<int>(nw);
     b.nle = c.take<int>(nw);
     b.vlist = c.take<int>(nw * b.vcap);
+    b.dgroups = c.take<int4>((size_t)n_heads * b.scap);
+    b.ndgroups = c.take<int>(n_heads);
+    b.diag_ml = c.take<float2>((size_t)n_heads * n);
+    b.diag_o = c.take<float>((size_t)n_heads * n * kD);
     return b;
 }
 
@@ -303,7 +310,7 @@ cudaError_t encode_attn_maps(AttnParams &P, const void *q, const void *k, const 
 
 int reset_counters(void *ws, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(static_cast<char *>(ws) + offsetof(WsHeader, tiles), 0,
-                                    2 * sizeof(unsigned long long), st);
+                                    sizeof(WsHeader) - offsetof(WsHeader, tiles), st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "cudaMemsetAsync");
 }
 
@@ -352,13 +359,45 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
                     bool slot_is_id, cudaStream_t st, bool tiles = false) {
     Carver cv(scratch, 0);
     VsPlanBufs b = carve_vs_plan(cv, c.n, c.n_heads, nv, ns);
-    cudaError_t e = run_vs_plan(b, v_idx, nv, s_idx, ns, c.n, c.n_heads, qtiles(c.n), st);
+    // whole slash tiles attend every key of a computed range: no CUDA-core pass
+    const float ratio = tiles ? 0.f : g_vs_diag_ratio.load();
+    cudaError_t e = run_vs_plan(b, v_idx, nv, s_idx, ns, c.n, c.n_heads, qtiles(c.n), ratio, st);
     if (e != cudaSuccess) return cuda_fail(e, "vs plan launch");
     AttnParams P;
     memset(&P, 0, sizeof(P));
     fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
     e = encode_attn_maps(P, q, k, v, c);
     if (e != cudaSuccess) return cuda_fail(e, "tensor map");
+    if (ratio > 0.f) {
+        // the sparse slash groups first, on the CUDA cores; the tile kernel merges their state
+        DiagParams D;
+        memset(&D, 0, sizeof(D));
+        D.tmap_k = P.tmap_k;
+        D.tmap_v = P.tmap_v;
+        D.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+        D.groups = b.dgroups;
+        D.ngroups = b.ndgroups;
+        D.gstride = b.scap;
+        D.offs = b.soff;
+        D.ostride = b.scap;
+        D.bits_v = b.bits_v;
+        D.bit_stride = b.stride;
+        D.ml = b.diag_ml;
+        D.o = b.diag_o;
+        D.hdr = P.hdr;
+        D.wait_limit_ns = P.wait_limit_ns;
+        D.n = c.n;
+        D.group = c.hq / c.hkv;
+        D.n_heads = c.n_heads;
+        D.n_qtiles = qtiles(c.n);
+        D.scale_log2 = P.scale_log2;
+        for (int i = 0; i < MINF_MAX_HEADS; ++i) D.head_ids[i] = P.head_ids[i];
+        e = run_vs_diag(D, st);
+        if (e != cudaSuccess) return cuda_fail(e, "vs sparse-slash launch");
+        P.vs_ndgroups = b.ndgroups;
+        P.vs_diag_ml = b.diag_ml;
+        P.vs_diag_o = b.diag_o;
+    }
     P.vs_groups = b.groups;
     P.vs_ngroups = b.ngroups;
     P.vs_gstride = b.scap;
@@ -793,7 +832,23 @@ int minf_stats(void *ws, minf_stream_t stream, uint64_t *tiles, uint64_t *pairs)
     return MINF_OK;
 }
 
+int minf_stats_detail(void *ws, minf_stream_t stream, uint64_t *out, int n_out) {
+    if (!ws || !out || n_out < 0) return fail(MINF_ERR_INVALID, "null argument");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    WsHeader h;
+    e = cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy stats");
+    const uint64_t v[7] = {h.tiles, h.pairs, h.pat_tiles[PAT_DENSE], h.pat_tiles[PAT_VS], h.pat_tiles[PAT_BLOCK],
+                           h.pat_tiles[PAT_ASHAPE], h.diag_pairs};
+    const int n = n_out < 7 ? n_out : 7;
+    for (int i = 0; i < n; ++i) out[i] = v[i];
+    return n;
+}
+
 void minf_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 2000000000ull); }
+
+void minf_set_vs_diag_ratio(float ratio) { g_vs_diag_ratio.store(ratio > 0.f ? ratio : 0.f); }
 
 int minf_check_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, minf_stream_t stream) {
     int rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES);

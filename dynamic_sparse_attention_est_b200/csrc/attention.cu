@@ -463,7 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (j + 2 < T && !issue_s(j + 2)) break;
             }
             umma_commit_warp(bar(B_ALL_DONE));  // always close: the epilogue (or the abort path) waits on it
-            if (P.hdr && lane == 0) atomicAdd(&P.hdr->tiles, (unsigned long long)T);
+            if (P.hdr && lane == 0) {
+                atomicAdd(&P.hdr->tiles, (unsigned long long)T);
+                atomicAdd(&P.hdr->pat_tiles[PAT], (unsigned long long)T);
+            }
         }
     } else {
         // ---------------------------------------------------------- softmax warpgroups
@@ -596,12 +599,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (ok) {
             tc_fence_after();
             const float2 s0 = ex[r], s1 = ex[128 + r];
-            const float m = fmaxf(s0.x, s1.x);
+            // a third partial state: the row's sparse-slash pairs, from the CUDA-core pass
+            float2 s2 = make_float2(-INFINITY, 0.f);
+            if constexpr (PAT == PAT_VS) {
+                if (P.vs_diag_ml && q < P.n && P.vs_ndgroups[hp] > 0) s2 = P.vs_diag_ml[(size_t)hp * P.n + q];
+            }
+            const bool has2 = s2.y > 0.f;
+            const float m = fmaxf(fmaxf(s0.x, s1.x), has2 ? s2.x : -INFINITY);
             const float a0 = s0.x == -INFINITY ? 0.f : ex2_approx(s0.x - m);
             const float a1 = (T < 2 || s1.x == -INFINITY) ? 0.f : ex2_approx(s1.x - m);
-            const float l = s0.y * a0 + s1.y * a1;
+            const float a2 = has2 ? ex2_approx(s2.x - m) : 0.f;
+            const float l = s0.y * a0 + s1.y * a1 + s2.y * a2;
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+            const float w0 = a0 * inv_l, w1 = a1 * inv_l, w2 = a2 * inv_l;
+            const float4 *o2 = has2 ? reinterpret_cast<const float4 *>(P.vs_diag_o + ((size_t)hp * P.n + q) * kD + wg * 64)
+                                    : nullptr;
             const size_t orow = (size_t)P.out_slot[hp] * P.n + min(q, P.n - 1);
             uint4 *dst = reinterpret_cast<uint4 *>(P.out + orow * kD + wg * 64);
             const uint32_t tO0 = tmem + lane_off + 256 + wg * 64, tO1 = tmem + lane_off + 384 + wg * 64;
@@ -623,13 +635,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     for (int e = 0; e < 32; ++e) o1[e] = 0u;
                 }
                 if (q < P.n) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o0[e] = __float_as_uint(__uint_as_float(o0[e]) * w0 + __uint_as_float(o1[e]) * w1);
+                    if (o2) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {  // columns 32 c + 4 i .. + 3 of this warpgroup's 64
+                            const float4 x = __ldg(o2 + c * 8 + i);
+                            o0[4 * i] = __float_as_uint(fmaf(x.x, w2, __uint_as_float(o0[4 * i])));
+                            o0[4 * i + 1] = __float_as_uint(fmaf(x.y, w2, __uint_as_float(o0[4 * i + 1])));
+                            o0[4 * i + 2] = __float_as_uint(fmaf(x.z, w2, __uint_as_float(o0[4 * i + 2])));
+                            o0[4 * i + 3] = __float_as_uint(fmaf(x.w, w2, __uint_as_float(o0[4 * i + 3])));
+                        }
+                    }
                     uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float v0 = __uint_as_float(o0[2 * e]) * w0 + __uint_as_float(o1[2 * e]) * w1;
-                        const float v1 = __uint_as_float(o0[2 * e + 1]) * w0 + __uint_as_float(o1[2 * e + 1]) * w1;
-                        pk[e] = pack_bf16x2(v0, v1);
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(o0[2 * e]), __uint_as_float(o0[2 * e + 1]));
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
@@ -748,12 +770,19 @@ __device__ int block_extract_bits(const uint32_t *bm, int words, int *out, int c
 // whose 128-row key ranges touch (consecutive offsets at most 128 apart).  A
 // group starts at an offset more than 128 past its predecessor and ends at
 // one more than 128 short of its successor; the j-th start and the j-th end
-// bound group j.
-__global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint32_t *bits_v, const uint32_t *bits_s,
+// bound group j.  Each group then goes to one of two paths: the tile kernel
+// (dense 128x128 tiles over the group's key range, masked per element) or the
+// CUDA-core pass (one pair per row and offset), whichever computes it for less:
+// a tile half costs about `diag_ratio` offsets of the CUDA-core pass, so a
+// group of m offsets whose range needs H halves goes there when
+// m < diag_ratio * H (0 sends every group to the tile kernel).  The offsets of
+// those groups are cleared from the slash bitmap, which from then on masks the
+// tile kernel's ranges.
+__global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint32_t *bits_v, uint32_t *bits_s,
                                                                      int words, int stride, int *vsorted, int *nvs,
-                                                                     int vcap,
-                                                                     int *soff, int scap, int2 *groups,
-                                                                     int *ngroups) {
+                                                                     int vcap, int *soff, int scap, int2 *groups,
+                                                                     int *ngroups, int4 *dgroups, int *ndgroups,
+                                                                     float diag_ratio) {
     __shared__ TopkShared sh;
     const int hp = blockIdx.x;
     const int cv = block_extract_bits<kExtractThreads>(bits_v + (size_t)hp * stride, words,
@@ -762,7 +791,7 @@ __global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint3
                                                        soff + (size_t)hp * scap, scap, sh);
     __syncthreads();  // the offsets written above are read by other threads below
     const int *so = soff + (size_t)hp * scap;
-    int2 *gr = groups + (size_t)hp * scap;
+    int4 *all = dgroups + (size_t)hp * scap;  // every group: (first offset, last offset, first index, last index)
     int n_start = 0, n_end = 0;
     for (int e0 = 0; e0 < cs; e0 += kExtractThreads) {
         const int e = e0 + (int)threadIdx.x;
@@ -774,14 +803,51 @@ __global__ void __launch_bounds__(kExtractThreads) vs_extract_kernel(const uint3
         }
         int tot;
         const int packed = block_excl_scan<kExtractThreads>(start | (end << 16), &tot, sh);
-        if (start) gr[n_start + (packed & 0xffff)].x = x;
-        if (end) gr[n_end + (packed >> 16)].y = x;
+        if (start) {
+            all[n_start + (packed & 0xffff)].x = x;
+            all[n_start + (packed & 0xffff)].z = e;
+        }
+        if (end) {
+            all[n_end + (packed >> 16)].y = x;
+            all[n_end + (packed >> 16)].w = e;
+        }
         n_start += tot & 0xffff;
         n_end += tot >> 16;
     }
+    __syncthreads();  // every group's four fields are written
+    int2 *tg = groups + (size_t)hp * scap;
+    uint32_t *bs = bits_s + (size_t)hp * stride;
+    int n_tile = 0, n_diag = 0;
+    for (int i0 = 0; i0 < n_start; i0 += kExtractThreads) {
+        const int i = i0 + (int)threadIdx.x;
+        int4 gd = make_int4(0, 0, 0, 0);
+        int to_tile = 0, to_diag = 0;
+        if (i < n_start) {
+            gd = all[i];
+            const int m = gd.w - gd.z + 1;
+            const int halves = (gd.y - gd.x + kTileM + kHalf - 1) / kHalf;
+            to_diag = diag_ratio > 0.f && (float)m < diag_ratio * (float)halves;
+            to_tile = !to_diag;
+        }
+        int tot;
+        // every read of this sweep happens before the scan's barriers, and the
+        // CUDA-core groups are compacted in place towards lower indices
+        const int packed = block_excl_scan<kExtractThreads>(to_tile | (to_diag << 16), &tot, sh);
+        if (to_tile) tg[n_tile + (packed & 0xffff)] = make_int2(gd.x, gd.y);
+        if (to_diag) {
+            all[n_diag + (packed >> 16)] = make_int4(gd.x, gd.y, gd.z, gd.w - gd.z + 1);
+            for (int j = gd.z; j <= gd.w; ++j) {
+                const int x = so[j];
+                atomicAnd(bs + (x >> 5), ~(1u << (x & 31)));
+            }
+        }
+        n_tile += tot & 0xffff;
+        n_diag += tot >> 16;
+    }
     if (threadIdx.x == 0) {
         nvs[hp] = cv;
-        ngroups[hp] = n_start;
+        ngroups[hp] = n_tile;
+        ndgroups[hp] = n_diag;
     }
 }
 
@@ -856,6 +922,9 @@ cudaError_t launch_attn(const AttnParams &P, cudaStream_t st) {
     if (fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
     const int grid = P.n_heads * P.n_qtiles;
     if (grid == 0) return cudaSuccess;
+    static const char *const names[] = {"attn_kernel<DENSE>", "attn_kernel<VS>", "attn_kernel<BLOCK>",
+                                        "attn_kernel<ASHAPE>"};
+    ProfScope prof(names[PAT], st);
     attn_kernel<PAT><<<grid, kThreads, kSmemBytes, st>>>(P);
     return cudaGetLastError();
 }
@@ -895,13 +964,15 @@ cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st) {
 cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_heads, int n_qtiles, int nb,
                         int *plan, int *cnt, int stride, cudaStream_t st) {
     const int nw = n_heads * n_qtiles;
+    ProfScope prof("bs_plan", st);
     bs_plan_kernel<<<(nw + 127) / 128, 128, 0, st>>>(blk_idx, blk_cnt, topk, n_heads, n_qtiles, nb, plan, cnt,
                                                      stride);
     return cudaGetLastError();
 }
 
 cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, const int *s_idx, int n_slash,
-                        int n, int n_heads, int n_qtiles, cudaStream_t st) {
+                        int n, int n_heads, int n_qtiles, float diag_ratio, cudaStream_t st) {
+    ProfScope prof("vs_plan", st);
     // the guards are cleared with the bitmaps
     const size_t bytes = sizeof(uint32_t) * (size_t)n_heads * b.stride;
     cudaError_t e = cudaMemsetAsync(b.bits_v - kBitGuard, 0, bytes, st);
@@ -909,7 +980,8 @@ cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, c
     if (e != cudaSuccess) return e;
     vs_mark_kernel<<<n_heads, 256, 0, st>>>(v_idx, n_vertical, s_idx, n_slash, n, b.bits_v, b.bits_s, b.stride);
     vs_extract_kernel<<<n_heads, kExtractThreads, 0, st>>>(b.bits_v, b.bits_s, b.words, b.stride, b.vsorted, b.nvs,
-                                                           b.vcap, b.soff, b.scap, b.groups, b.ngroups);
+                                                           b.vcap, b.soff, b.scap, b.groups, b.ngroups, b.dgroups,
+                                                           b.ndgroups, diag_ratio);
     const int nw = n_heads * n_qtiles;
     vs_workitem_kernel<<<(nw + 3) / 4, 128, 0, st>>>(b.vsorted, b.nvs, b.vcap, b.groups, b.ngroups, b.scap,
                                                      b.bits_s, b.stride, n, n_heads, n_qtiles, b.nsh, b.nvert,

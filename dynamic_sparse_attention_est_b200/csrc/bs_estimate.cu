@@ -157,6 +157,7 @@ cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStrea
     HeadList hl;
     for (int i = 0; i < MINF_MAX_HEADS; ++i) hl.ids[i] = i < a.n_heads ? a.head_ids[i] : 0;
     // pooled Q of the listed heads, pooled K of every kv-head
+    ProfScope prof("bs_estimate (pool, scores, top-k)", st);
     const int warps = a.n_heads * nb;
     pool_kernel<<<(warps + 7) / 8, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(a.q), hl, true, a.n_heads,
                                                  a.n, b.qp);

@@ -25,6 +25,8 @@ struct WsHeader {
     int site;  // where the first bounded wait gave up: role << 24 | barrier << 16 | tile
     unsigned long long tiles;
     unsigned long long pairs;
+    unsigned long long pat_tiles[4];  // tiles by attention kernel pattern (PAT_*)
+    unsigned long long diag_pairs;    // pairs of the CUDA-core sparse-slash pass (included in pairs)
 };
 static_assert(sizeof(WsHeader) <= MINF_STATUS_BYTES, "header fits the status block");
 
@@ -75,6 +77,12 @@ struct AttnParams {
     const uint32_t *vs_bits_s;  // per head: bitmap of slash offsets (head hp at hp * bit_stride)
     const uint32_t *vs_bits_v;  // per head: bitmap of vertical keys
     int bit_stride;             // words per head, kBitGuard zero words on each side included
+    // Vertical-Slash pairs of the sparse slash groups, computed beforehand on the
+    // CUDA cores (null: none): per query row of each listed head, (m, l) in the
+    // log2 domain and the unnormalised O, merged in the epilogue
+    const int *vs_ndgroups;     // per head: its number of such groups (0: nothing to merge)
+    const float2 *vs_diag_ml;   // [n_heads][n]
+    const float *vs_diag_o;     // [n_heads][n][128], read only where l > 0
     int head_ids[MINF_MAX_HEADS];
     int out_slot[MINF_MAX_HEADS];  // output row block of each listed head (its position, or its id)
     // Launch order: the listed heads in n_kvgroups groups, taken one group after
@@ -84,6 +92,27 @@ struct AttnParams {
     int n_kvgroups;
     int kv_order[MINF_MAX_HEADS];       // head positions sorted by kv-head
     int kv_start[MINF_MAX_HEADS + 1];   // kv_order index where each group starts
+};
+
+// The CUDA-core pass over the sparse slash groups of Vertical-Slash.
+struct DiagParams {
+    CUtensorMap tmap_k;  // [hkv][n][128], box {64, 64, 1}, 128B swizzle
+    CUtensorMap tmap_v;
+    const __nv_bfloat16 *q;
+    const int4 *groups;       // per head: (first offset, last offset, index of the first in offs, count), ascending
+    const int *ngroups;       // per head
+    int gstride;
+    const int *offs;          // per head: the sorted distinct slash offsets
+    int ostride;
+    const uint32_t *bits_v;   // per head: bitmap of vertical keys
+    int bit_stride;
+    float2 *ml;               // [n_heads][n] (m, l), log2 domain
+    float *o;                 // [n_heads][n][128] unnormalised, written where l > 0
+    WsHeader *hdr;
+    unsigned long long wait_limit_ns;
+    int n, group, n_heads, n_qtiles;
+    float scale_log2;
+    int head_ids[MINF_MAX_HEADS];
 };
 
 // Bits [start, start + 64) of a bitmap of nbits bits; positions outside

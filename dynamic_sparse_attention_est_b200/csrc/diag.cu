@@ -1,0 +1,345 @@
+// diag.cu -- Vertical-Slash attention over sparse slash groups, on the CUDA cores.
+//
+// A slash line is the diagonal of the attention matrix at a fixed offset o:
+// query i meets key i - o (AICon talk "以 KV 缓存为中心的高效长文本方法", the
+// vertical and slash observation).  Where the estimated offsets are dense, the
+// tensor-core kernel computes their key ranges as whole 128x128 tiles and masks
+// them (news article "单卡A100实现百万token推理…", Figure 4: slashes as dense
+// blocks).  Where they are sparse -- an offset alone, or a few within 128 of one
+// another -- a 128-row query tile meets each offset in only one key per row, and
+// a 128x128 tile wastes 127 of every 128 products and exponentials.  This kernel
+// takes those groups instead: for each query tile it stages the groups' key
+// ranges in 64-key chunks (K and V, by TMA, as the tile kernel does), and each
+// query row computes only its in-mask pairs, one dot product, one exponential
+// and one V update per offset, in fp32 with bf16 operands.
+//
+// It produces a partial softmax state per query row over exactly those pairs
+// (each slash pair whose key is not a vertical key; verticals belong to the tile
+// kernel) -- the running max m and sum l in the log2 domain and the unnormalised
+// O -- which the tile kernel merges into its own in its epilogue.
+//
+// Roles (288 threads, one persistent CTA per SM striding over the work items):
+//   warps 0..7  consumers: two threads per query row (lane l of warp w holds row
+//               16 w + (l & 15) and head dims [64 (l >> 4), 64 (l >> 4) + 64))
+//   warp 8      TMA producer: one 64-key chunk of K and V per stage, 6 stages
+// A chunk stays until every consumer warp has moved past it; each warp releases
+// chunks in order, after it has seen them full.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace minf {
+
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kDiagThreads = (kConsumerWarps + 1) * 32;
+constexpr int kDiagStages = 6;
+constexpr uint32_t kChunkBytes = 32768;  // 64 keys x 128 dims x 2 B, K then V
+constexpr uint32_t kDiagSmem = kDiagStages * kChunkBytes + 256 + 1024;  // + barriers + alignment slack
+
+// acc + lo(a) lo(b) + hi(a) hi(b): bf16 operands, fp32 products and sums (one
+// rounding per fused multiply-add, as an fp32 FMA of the widened operands).
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "=f"(r)
+        : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+
+// (o0, o1) += p * (lo(v), hi(v)) with p and v bf16, o fp32.
+__device__ __forceinline__ void axpy2_bf16(uint32_t v, uint16_t p, float &o0, float &o1) {
+    asm("{\n\t.reg .b16 vl, vh;\n\t"
+        "mov.b32 {vl, vh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, %3, vl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, %3, vh, %1;\n\t}"
+        : "+f"(o0), "+f"(o1)
+        : "r"(v), "h"(p));
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+    return v;
+}
+
+// Warp-wide TMA load of one chunk: keys [y, y + 64) of kv-head z, K into
+// dst[0, 16K) and V into dst[16K, 32K), each as two 64-column 128B-swizzled
+// boxes.  Every lane calls it with the same operands; elect.sync picks the
+// lane that adds the 32 KB to `bar` and issues the four loads.
+__device__ __forceinline__ void tma_load_kv_chunk_warp(uint32_t dst, const void *tmap_k, const void *tmap_v,
+                                                       uint32_t bar, int y, int z) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%2], 32768;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {0, %4, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%6], [%1, {64, %4, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%7], [%3, {0, %4, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%8], [%3, {64, %4, %5}], [%2];\n\t}\n" ::"r"(dst),
+        "l"(tmap_k), "r"(bar), "l"(tmap_v), "r"(y), "r"(z), "r"(dst + 8192), "r"(dst + 16384), "r"(dst + 24576)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_constant__ DiagParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t ring = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDiagStages * kChunkBytes);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kDiagStages);
+    auto full_bar = [&](int s) { return smem_u32(bars + s); };
+    auto empty_bar = [&](int s) { return smem_u32(bars + kDiagStages + s); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDiagStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const WaitCtl wc{abort_flag, P.hdr ? &P.hdr->status : nullptr, P.wait_limit_ns};
+    const int n_items = P.n_heads * P.n_qtiles;
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&P.tmap_k);
+            tma_prefetch_desc(&P.tmap_v);
+        }
+        __syncwarp();
+        int c = 0;  // chunks issued by this CTA, over all its work items
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            // heaviest query tiles first (a tile meets every offset at or below its last row)
+            const int t = P.n_qtiles - 1 - it / P.n_heads, hp = it % P.n_heads;
+            const int ng = P.ngroups[hp];
+            const int4 *groups = P.groups + (size_t)hp * P.gstride;
+            const int g = P.head_ids[hp] / P.group;
+            const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, P.n - 1);
+            for (int gi = 0; ok && gi < ng; ++gi) {
+                const int4 G = __ldg(groups + gi);
+                if (G.x > rmax) break;  // groups ascend: no row of this tile reaches the rest
+                const int a = max(0, r0 - G.y), b = rmax - G.x;
+                const int nc = (b - a + kHalf) / kHalf;
+                for (int j = 0; j < nc; ++j, ++c) {
+                    const int s = c % kDiagStages;
+                    const bool got = wait_bounded(empty_bar(s), ((c / kDiagStages) & 1) ^ 1, wc, wait_site(8, s, c));
+                    if (!__all_sync(0xffffffffu, got)) {
+                        ok = false;
+                        break;
+                    }
+                    tma_load_kv_chunk_warp(ring + s * kChunkBytes, &P.tmap_k, &P.tmap_v, full_bar(s), a + j * kHalf,
+                                           g);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full_bar(s));
+                }
+            }
+        }
+        if (*abort_flag && lane == 0) {
+            // drain: let the loads already issued land before the CTA exits
+            volatile int no_abort = 0;
+            const WaitCtl drain{&no_abort, nullptr, 50000000ull};
+            for (int j = max(0, c - kDiagStages); j < c; ++j)
+                wait_bounded(full_bar(j % kDiagStages), (j / kDiagStages) & 1, drain);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int rw = warp * 16;           // first row of this warp
+    const int r = rw + (lane & 15);     // query row in the tile
+    const int hf = lane >> 4;           // head-dimension half
+    const float sl2 = P.scale_log2;
+    const uint32_t kbase = ring + hf * 8192, vbase = ring + 16384 + hf * 8192;
+    int c_base = 0;  // sequence number of the current group's first chunk
+    int got = 0;     // chunks [0, got) seen full by this warp
+    int rel = 0;     // chunks [0, rel) released by this warp
+    bool ok = true;
+    unsigned long long pairs = 0;
+    auto see = [&]() -> bool {  // waits for chunk `got` to be full (warp-uniform)
+        const int s = got % kDiagStages;
+        const bool gfull = wait_bounded(full_bar(s), (got / kDiagStages) & 1, wc, wait_site(9, s, got));
+        if (!__all_sync(0xffffffffu, gfull)) return false;
+        ++got;
+        return true;
+    };
+    auto release = [&]() {  // chunk `rel`, seen full and no longer needed
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(rel % kDiagStages));
+        ++rel;
+    };
+    // From now on this warp needs chunks [lo, hi] (at most two; hi < lo at a group's
+    // end).  Everything below lo is released first -- chunks not seen yet are seen
+    // and released one by one -- so a warp never waits for a chunk while holding one
+    // it no longer needs; the ring then always has room for the chunk awaited by
+    // the warp that is furthest behind.
+    auto need = [&](int lo, int hi) -> bool {
+        while (rel < lo && rel < got) release();
+        while (got < lo) {
+            if (!see()) return false;
+            release();
+        }
+        while (got <= hi)
+            if (!see()) return false;
+        return true;
+    };
+    for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        const int t = P.n_qtiles - 1 - it / P.n_heads, hp = it % P.n_heads;
+        const int ng = P.ngroups[hp];
+        if (ng == 0) continue;  // the tile kernel reads no state for this head
+        const int h = P.head_ids[hp];
+        const int4 *groups = P.groups + (size_t)hp * P.gstride;
+        const int *offs = P.offs + (size_t)hp * P.ostride;
+        const uint32_t *bv = P.bits_v + (size_t)hp * P.bit_stride;
+        const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, P.n - 1);
+        const int qi = r0 + r;
+        const bool row_ok = qi <= rmax;
+        const int last_r = rmax - r0;  // last valid row of the tile
+        uint32_t qv[32];
+        {
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(P.q + ((size_t)h * P.n + min(qi, P.n - 1)) * kD + hf * 64);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 x = row_ok ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+                qv[4 * i] = x.x;
+                qv[4 * i + 1] = x.y;
+                qv[4 * i + 2] = x.z;
+                qv[4 * i + 3] = x.w;
+            }
+        }
+        float o[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) o[e] = 0.f;
+        float m = -INFINITY, l = 0.f;
+        for (int gi = 0; ok && gi < ng; ++gi) {
+            const int4 G = __ldg(groups + gi);
+            if (G.x > rmax) break;
+            const int a = max(0, r0 - G.y), b = rmax - G.x;
+            const int nc = (b - a + kHalf) / kHalf;
+            // offsets of the group from the largest down: the key ranges move forward
+            for (int j = G.w - 1; j >= 0; --j) {
+                const int off = __ldg(offs + G.z + j);
+                const int u0 = r0 - off - a;  // range position of row 0's key
+                const int ulo = max(0, u0 + rw), uhi = min(u0 + rw + 15, u0 + last_r);
+                if (ulo > uhi) continue;  // no valid row of this warp meets a key of this offset
+                if (!need(c_base + (ulo >> 6), c_base + (uhi >> 6))) {
+                    ok = false;
+                    break;
+                }
+                const int u = u0 + r;
+                bool use = row_ok && u >= 0;
+                if (use) {
+                    const int key = a + u;
+                    use = !((__ldg(bv + (key >> 5)) >> (key & 31)) & 1u);  // verticals are the tile kernel's
+                }
+                float s = 0.f;
+                uint32_t row_off = 0;
+                int sw = 0;
+                if (use) {
+                    const int ur = u & 63;
+                    row_off = (uint32_t)((c_base + (u >> 6)) % kDiagStages) * kChunkBytes + (uint32_t)ur * 128;
+                    sw = ur & 7;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint4 kk = lds128(kbase + row_off + ((i ^ sw) << 4));
+                        acc[0] = dot2_bf16(kk.x, qv[4 * i], acc[0]);
+                        acc[1] = dot2_bf16(kk.y, qv[4 * i + 1], acc[1]);
+                        acc[2] = dot2_bf16(kk.z, qv[4 * i + 2], acc[2]);
+                        acc[3] = dot2_bf16(kk.w, qv[4 * i + 3], acc[3]);
+                    }
+                    s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                }
+                s += __shfl_xor_sync(0xffffffffu, s, 16);  // the two halves of the row's dot product
+                if (use) {
+                    const float x = s * sl2;
+                    if (x > m + 8.0f) {  // the running max moves only when it grows by more than 2^8
+                        const float alpha = ex2_approx(m - x);  // 0 while m = -inf
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) o[e] *= alpha;
+                        l *= alpha;
+                        m = x;
+                    }
+                    const float p = ex2_approx(x - m);
+                    l += p;
+                    const uint16_t pb = bf16_bits(p);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint4 vv = lds128(vbase + row_off + ((i ^ sw) << 4));
+                        axpy2_bf16(vv.x, pb, o[8 * i], o[8 * i + 1]);
+                        axpy2_bf16(vv.y, pb, o[8 * i + 2], o[8 * i + 3]);
+                        axpy2_bf16(vv.z, pb, o[8 * i + 4], o[8 * i + 5]);
+                        axpy2_bf16(vv.w, pb, o[8 * i + 6], o[8 * i + 7]);
+                    }
+                    pairs += hf == 0;
+                }
+            }
+            if (!ok) break;
+            // the group's remaining chunks: seen full, then released
+            if (!need(c_base + nc, c_base + nc - 1)) {
+                ok = false;
+                break;
+            }
+            c_base += nc;
+        }
+        // the row's partial softmax state: (m, l) and the unnormalised O
+        if (ok && row_ok) {
+            const size_t row = (size_t)hp * P.n + qi;
+            if (hf == 0) P.ml[row] = make_float2(m, l);
+            if (l > 0.f) {
+                float4 *dst = reinterpret_cast<float4 *>(P.o + row * kD + hf * 64);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            }
+        }
+    }
+    if (P.hdr) {
+#pragma unroll
+        for (int sft = 16; sft > 0; sft >>= 1) pairs += __shfl_xor_sync(0xffffffffu, pairs, sft);
+        if (lane == 0 && pairs) {
+            atomicAdd(&P.hdr->pairs, pairs);
+            atomicAdd(&P.hdr->diag_pairs, pairs);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t run_vs_diag(const DiagParams &P, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(vs_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // persistent: one CTA per SM, each striding over the work items heaviest first
+    const int items = P.n_heads * P.n_qtiles;
+    const int grid = std::min(items, std::max(1, sms));
+    if (grid == 0) return cudaSuccess;
+    ProfScope prof("vs_diag_kernel", st);
+    vs_diag_kernel<<<grid, kDiagThreads, kDiagSmem, st>>>(P);
+    return cudaGetLastError();
+}
+
+}  // namespace minf

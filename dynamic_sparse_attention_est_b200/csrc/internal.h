@@ -9,6 +9,20 @@ namespace minf {
 
 struct AttnParams;
 
+// Launch timing (minf_profile_enable): while enabled, an event pair around the
+// scope's launches on `st`, read back by minf_profile_read.
+class ProfScope {
+  public:
+    ProfScope(const char *name, cudaStream_t st);
+    ~ProfScope();
+    ProfScope(const ProfScope &) = delete;
+    ProfScope &operator=(const ProfScope &) = delete;
+
+  private:
+    cudaStream_t st_;
+    cudaEvent_t end_;
+};
+
 // Device buffers of the Vertical-Slash tile plan (all inside the workspace).
 struct VsPlanBufs {
     uint32_t *bits_v, *bits_s;  // head hp's n bits at + hp * stride, kBitGuard zero words on each side
@@ -16,11 +30,15 @@ struct VsPlanBufs {
     int *vsorted, *nvs;         // [n_heads][vcap], [n_heads]
     int vcap;
     int *soff;                  // [n_heads][scap]
-    int2 *groups;               // [n_heads][scap]
+    int2 *groups;               // [n_heads][scap] slash groups of the tile kernel
     int *ngroups;               // [n_heads]
+    int4 *dgroups;              // [n_heads][scap] slash groups of the CUDA-core pass
+    int *ndgroups;              // [n_heads]
     int scap;
     int *nsh, *nvert, *nle;     // [n_work]
     int *vlist;                 // [n_work][vcap]
+    float2 *diag_ml;            // [n_heads][n] partial (m, l) of the CUDA-core pass
+    float *diag_o;              // [n_heads][n][128] its unnormalised O
 };
 
 // 3D TMA map over a bf16 [heads][n][128] tensor: box {64, 64, 1}, 128B swizzle.
@@ -30,7 +48,9 @@ cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st);
 cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_heads, int n_qtiles, int nb,
                         int *plan, int *cnt, int stride, cudaStream_t st);
 cudaError_t run_vs_plan(const VsPlanBufs &b, const int *v_idx, int n_vertical, const int *s_idx, int n_slash,
-                        int n, int n_heads, int n_qtiles, cudaStream_t st);
+                        int n, int n_heads, int n_qtiles, float diag_ratio, cudaStream_t st);
+struct DiagParams;
+cudaError_t run_vs_diag(const DiagParams &P, cudaStream_t st);
 
 // Vertical-Slash estimation.
 struct VsEstBufs {

@@ -41,7 +41,7 @@ constexpr uint32_t kSmemP = kSmemK + kStages * kTileBytes;  // 128 x kPStride fl
 constexpr uint32_t kSmemBar = (kSmemP + 128 * kPStride * 4 + 255) & ~255u;
 constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;
 
-enum : int { B_Q = 0, B_KF = 1, B_KE = 4, B_SF = 7, B_SE = 9, B_COUNT = 11 };
+enum : int { B_Q = 0, B_KF = 1, B_KE = 4, B_SF = 7, B_SE = 9, B_DONE = 11, B_COUNT = 12 };
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, false);
 
@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
             mbar_init(bar(B_SF + b), 1);
             mbar_init(bar(B_SE + b), 256);
         }
+        mbar_init(bar(B_DONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
             }
             // K tiles: the whole warp runs the loop (warp-uniform operands), one elected
             // lane issues each stage's loads
+            int issued = 0;
             for (int j = 0; j < T; ++j) {
                 const int s = j % kStages;
                 const bool got = wait_bounded(bar(B_KE + s), ((j / kStages) & 1) ^ 1, wc, wait_site(5, B_KE + s, j));
@@ -120,6 +122,15 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
                 tma_load_stage_warp(sK + s * kTileBytes, &P.tmap_k, bar(B_KF + s), kTileBytes, key0, key0 + 64, g, 3u);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_KF + s));
+                issued = j + 1;
+            }
+            if (*abort_flag && lane == 0) {
+                // drain: let the Q load and the K loads already issued land before the CTA exits
+                volatile int no_abort = 0;
+                const WaitCtl drain{&no_abort, nullptr, 50000000ull};
+                wait_bounded(bar(B_Q), 0, drain);
+                for (int j = max(0, issued - kStages); j < issued; ++j)
+                    wait_bounded(bar(B_KF + j % kStages), (j / kStages) & 1, drain);
             }
         }
     } else if (warp == 1) {
@@ -138,6 +149,13 @@ __global__ void __launch_bounds__(kThreads, 1) vs_est_kernel(const __grid_consta
                 umma_ss_tile_warp(tmem + b * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
                 umma_commit_warp(bar(B_KE + s));
                 umma_commit_warp(bar(B_SF + b));
+            }
+            if (*abort_flag) {
+                // the MMAs already issued complete before TMEM is freed
+                umma_commit_warp(bar(B_DONE));
+                volatile int no_abort = 0;
+                const WaitCtl drain{&no_abort, nullptr, 50000000ull};
+                wait_bounded(bar(B_DONE), 0, drain);
             }
         }
     } else if (warp >= 4) {
@@ -363,13 +381,17 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
         e = cudaFuncSetAttribute(vs_est_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = np * b.n_chunks;
-    vs_est_kernel<0><<<grid, kThreads, kSmemBytes, st>>>(P);
-    lse_combine_kernel<<<(np * 128 + 255) / 256, 256, 0, st>>>(b.part, np, b.n_chunks, b.lse2);
-    vs_est_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(P);
-    dim3 sg((a.n + 255) / 256, a.n_heads);
-    slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash, b.diag0);
+    {
+        ProfScope prof("vs_estimate (vs_est_kernel x2 + combines)", st);
+        vs_est_kernel<0><<<grid, kThreads, kSmemBytes, st>>>(P);
+        lse_combine_kernel<<<(np * 128 + 255) / 256, 256, 0, st>>>(b.part, np, b.n_chunks, b.lse2);
+        vs_est_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(P);
+        dim3 sg((a.n + 255) / 256, a.n_heads);
+        slash_combine_kernel<<<sg, 256, 0, st>>>(b.diag, a.n, b.n_ktiles, b.slash, b.diag0);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    ProfScope prof("vs_topk", st);
     const int *kv = nullptr, *ks = nullptr;
     if (a.topp) {
         // top-p: per-row counts by mass, then the same ordered selection with those counts

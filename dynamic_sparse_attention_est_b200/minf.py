@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
-from typing import Optional, Sequence, Tuple
+from typing import Dict, Optional, Sequence, Tuple
 
 import torch
 
@@ -58,7 +58,11 @@ _SIGS = {
     "minf_vs_estimate_noalloc_check_timeout": (_I, [_I, _U64, _P]),
     "minf_status": (_I, [_P, _P]),
     "minf_stats": (_I, [_P, _P, ctypes.POINTER(_U64), ctypes.POINTER(_U64)]),
+    "minf_stats_detail": (_I, [_P, _P, ctypes.POINTER(_U64), _I]),
     "minf_set_wait_limit_ns": (None, [_U64]),
+    "minf_set_vs_diag_ratio": (None, [ctypes.c_float]),
+    "minf_profile_enable": (None, [_I]),
+    "minf_profile_read": (_I, [ctypes.c_char_p, _SZ]),
     "minf_check_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
     "minf_selftest_exp2": (_I, [_P, _P, _P, _I, _P]),
     "minf_version": (ctypes.c_char_p, []),
@@ -337,8 +341,39 @@ def minf_stats(ws: torch.Tensor) -> Tuple[int, int]:
     return int(t.value), int(p.value)
 
 
+def minf_stats_detail(ws: torch.Tensor) -> Dict[str, int]:
+    """Counters of the last attention call on ws, split by kernel."""
+    arr = (_U64 * 7)()
+    n = lib().minf_stats_detail(_ptr(ws), _stream(ws.device), arr, 7)
+    if n < 0:
+        _check(n, "minf_stats_detail")
+    keys = ["tiles", "pairs", "tiles_dense", "tiles_vs", "tiles_block", "tiles_ashape", "diag_pairs"]
+    return {k: int(arr[i]) for i, k in enumerate(keys[:n])}
+
+
 def minf_set_wait_limit_ns(ns: int) -> None:
     lib().minf_set_wait_limit_ns(int(ns))
+
+
+def minf_set_vs_diag_ratio(ratio: float) -> None:
+    """Sparse slash groups of m offsets over H half-tiles go to the CUDA-core pass when m < ratio * H."""
+    lib().minf_set_vs_diag_ratio(float(ratio))
+
+
+def minf_profile_enable(on: bool = True) -> None:
+    lib().minf_profile_enable(1 if on else 0)
+
+
+def minf_profile_read() -> Dict[str, Tuple[int, float]]:
+    """{kernel name: (launches, total ms)} of the launches timed since the last read."""
+    n = int(lib().minf_profile_read(None, 0))
+    buf = ctypes.create_string_buffer(n + 1)
+    lib().minf_profile_read(buf, n + 1)
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, cnt, ms = line.split("\t")
+        out[name] = (int(cnt), float(ms))
+    return out
 
 
 def minf_check_wait_timeout(ws: torch.Tensor, limit_ns: int) -> None:

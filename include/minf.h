@@ -253,11 +253,35 @@ int minf_status(void *ws, minf_stream_t stream);
 int minf_stats(void *ws, minf_stream_t stream, uint64_t *tiles, uint64_t *pairs);
 
 /*
+ * The same counters split by kernel (no counterpart in the method's sources):
+ * writes min(n_out, 7) values to the host array out -- tiles, pairs, then the
+ * tiles of the dense, Vertical-Slash, Block-Sparse and A-shape (Tri-shape
+ * included) attention kernels, then the pairs computed by the CUDA-core
+ * sparse-slash pass (part of pairs) -- and returns how many it wrote.
+ */
+int minf_stats_detail(void *ws, minf_stream_t stream, uint64_t *out, int n_out);
+
+/*
  * Sets the limit, in nanoseconds, after which a device-side wait gives up and
  * records MINF_ERR_TIMEOUT (default 2e9 ns; 0 restores the default).  Applies
  * to launches made after the call, process-wide.
  */
 void minf_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Routing of Vertical-Slash slash groups (a tuning knob; the method's sources
+ * compute every slash as dense blocks, [NEWS] Figure 4).  Offsets at most 128
+ * apart form a group whose key range a 128-row query tile computes as H
+ * half-tiles of 64 keys on the tensor cores, masked per element.  A group of m
+ * offsets goes instead to a CUDA-core pass that computes only the m in-mask
+ * pairs of each query row (one dot product, one exponential and one V update
+ * per offset) when m < ratio * H.  The result is the same token-exact masked
+ * softmax either way (the two partial states are merged per row); only the
+ * time differs.  ratio <= 0 sends every group to the tensor cores.  Default
+ * 2.0; applies to minf_vs_attention and the mixed layer (not to
+ * minf_vs_attention_tiles), process-wide, for calls made after it.
+ */
+void minf_set_vs_diag_ratio(float ratio);
 
 /*
  * Failure-detection self-test: launches one kernel whose wait nothing will
@@ -317,6 +341,20 @@ int minf_vs_estimate_noalloc_status(int device, minf_stream_t stream);
  * block, as a timed-out estimate would.  Asynchronous on `stream`.
  */
 int minf_vs_estimate_noalloc_check_timeout(int device, uint64_t limit_ns, minf_stream_t stream);
+
+/*
+ * Launch timing (no counterpart in the method's sources; for measuring this
+ * library): while enabled (on != 0), every attention, estimate and plan launch
+ * sequence of the library is bracketed by two CUDA events on the stream it
+ * runs on.  minf_profile_read waits for the recorded events, writes one line
+ * per kernel name -- "name<TAB>launches<TAB>total milliseconds" -- into the
+ * host buffer buf (at most len bytes, NUL-terminated), clears the records and
+ * returns the length of the full text (larger than len - 1 if it was cut).
+ * With buf NULL it only returns that length and keeps the records.
+ * Do not read while calls of the library are being made on other threads.
+ */
+void minf_profile_enable(int on);
+int minf_profile_read(char *buf, size_t len);
 
 /* Library version string and the message of the last host-side error. */
 const char *minf_version(void);

@@ -25,7 +25,10 @@ def test_estimate_bytes_per_workload(name):
 def test_parse_defaults_and_options(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py"])
     a = bench.parse()
-    assert (a.gpus, a.workload, a.impl, a.vs_mode, a.shard, a.topp) == (1, "vs-gqa-32k", "minf", "exact", "layers", None)
+    assert (a.gpus, a.workload, a.impl, a.vs_mode, a.shard, a.topp) == (1, "mixed-gqa-1m", "minf", "exact", "layers", None)
+    assert a.steps == 5 and a.cpu_mode == "auto"
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "vs-gqa-32k"])
+    assert bench.parse().steps == 20
     monkeypatch.setattr(sys, "argv", ["bench.py", "--vs-mode", "tiles", "--topp", "0.9", "--shard", "heads"])
     a = bench.parse()
     assert (a.vs_mode, a.topp, a.shard) == ("tiles", 0.9, "heads")
@@ -63,3 +66,22 @@ def test_bf16_peak_choice():
     assert bench.pick_bf16_peak(peaks, 200.0, {"sm_mhz": None, "reasons": ["sw_power_cap"]})[1] == "bf16_tflops_sustained"
     assert bench.pick_bf16_peak(peaks, 9000.0, None)[1] == "bf16_tflops_sustained"
     assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, 9000.0, capped) == (1590.0, "bf16_tflops")
+
+
+def test_cpu_sample_projects_every_pattern_of_a_mixed_layer(orc):
+    """The bounded CPU sample of a mixed layer times each pattern present and says it
+    is a projection; at a small size the full layer is timed instead."""
+    import dataclasses
+
+    w = dataclasses.replace(synth.WORKLOADS["mixed-gqa-1m"], n=4096, hq=8, hkv=2, n_vertical=64, n_slash=128,
+                            topk=8, window=512)
+    pats = synth.mixed_head_patterns(w, seed=0)
+    x = synth.generate(w, seed=0, device="cpu", hq=1, hkv=1)
+    r = bench.cpu_sample(w, x, orc, 0.5, pats=pats)
+    assert r["projected"] and r["value"] > 0 and r["cores"] >= 1
+    for p in set(pats):
+        assert f"{p} x{pats.count(p)}" in r["sample"]
+    wv = dataclasses.replace(synth.WORKLOADS["vs-gqa-32k"], n=1024, hq=2, hkv=1, n_vertical=32, n_slash=64)
+    xf = synth.generate(wv, seed=1, device="cpu")
+    rf = bench.cpu_sample(wv, xf, orc, 0.5, full=True)
+    assert not rf["projected"] and rf["value"] > 0 and "timed" in rf["sample"]

@@ -497,3 +497,90 @@ def test_repeat_runs_bit_identical():
     for name, a, b in zip(names, first, second):
         assert torch.equal(a.view(torch.uint8) if a.dtype == torch.bfloat16 else a,
                            b.view(torch.uint8) if b.dtype == torch.bfloat16 else b), f"{name} differs between runs"
+
+
+# ----------------------------------------------------------------------------- sparse slash groups
+def _sparse_vs_indices(rng, n, nh, nv, n_far):
+    """Verticals anywhere; slash offsets mostly far apart (lone offsets), some in
+    pairs and triples within 128 of each other, offset 0 and one past n."""
+    vi = np.full((nh, nv), -1, np.int32)
+    si = np.full((nh, 3 * n_far + 2), -1, np.int32)
+    for hp in range(nh):
+        vi[hp] = rng.choice(n, nv, replace=False)
+        base = np.sort(rng.choice(np.arange(1, n), n_far, replace=False))
+        extra = [b + rng.integers(1, 100) for b in base[::3]] + [b + rng.integers(1, 60) for b in base[::5]]
+        offs = np.unique(np.concatenate([[0], base, extra, [n + 5]]))
+        si[hp, :len(offs)] = rng.permutation(offs)
+    return vi, si
+
+
+@pytest.mark.parametrize("n,hq,hkv,nv,n_far", [(4160, 2, 1, 40, 24), (8192, 4, 2, 100, 60), (1088, 1, 1, 8, 6)])
+def test_vs_sparse_slash_groups_cuda_core_path(orc, n, hq, hkv, nv, n_far):
+    """Lone and small slash groups take the CUDA-core pass (the default routing), the
+    rest the tile kernel; verticals that lie on those diagonals count once.  Both
+    routings agree with the oracle on the same indices."""
+    q, k, v = inputs(n, hq, hkv, seed=n + nv)
+    vi, si = _sparse_vs_indices(np.random.default_rng(n), n, hq, nv, n_far)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    qc, kc, vc = cuda(q, k, v)
+    vt, st = torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda()
+    ws = minf.workspace(minf.workspace_bytes(minf.OP_VS_ATTENTION, hq, hkv, n, hq, vi.shape[1], si.shape[1]),
+                        qc.device)
+    try:
+        for ratio in (2.0, 0.0, 1000.0):  # default, tensor cores only, CUDA cores for every group
+            minf.minf_set_vs_diag_ratio(ratio)
+            out, lse = minf.minf_vs_attention(qc, kc, vc, vt, st, scale=SCALE, ws=ws)
+            check_attention(out, lse, ref, rl, f"VS sparse groups n={n} ratio={ratio}")
+            tiles, pairs = minf.minf_stats(ws)
+            assert minf.minf_status(ws) == minf.MINF_OK
+            # every in-mask pair is counted once, by one of the two paths
+            assert pairs == _mask_pairs(vi, si, n), (ratio, pairs)
+    finally:
+        minf.minf_set_vs_diag_ratio(2.0)
+
+
+def _mask_pairs(vi, si, n):
+    """Number of (query, key) pairs of the Vertical-Slash mask, counted from its definition."""
+    total = 0
+    for hp in range(vi.shape[0]):
+        vset = np.zeros(n, bool)
+        vset[vi[hp][(vi[hp] >= 0) & (vi[hp] < n)]] = True
+        sset = np.unique(si[hp][(si[hp] >= 0) & (si[hp] < n)])
+        for i in range(n):
+            keys = np.zeros(i + 1, bool)
+            keys |= vset[:i + 1]
+            o = sset[sset <= i]
+            keys[i - o] = True
+            total += int(keys.sum())
+    return total
+
+
+def test_vs_sparse_groups_head_subset_and_determinism(orc):
+    """A listed head subset through the CUDA-core pass, twice: bit-identical results."""
+    n, hq, hkv = 2112, 8, 2
+    q, k, v = inputs(n, hq, hkv, seed=41)
+    ids = [6, 1, 3]
+    vi, si = _sparse_vs_indices(np.random.default_rng(41), n, len(ids), 30, 20)
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si, head_ids=ids)
+    qc, kc, vc = cuda(q, k, v)
+    vt, st = torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda()
+    o1, l1 = minf.minf_vs_attention(qc, kc, vc, vt, st, scale=SCALE, head_ids=ids)
+    check_attention(o1, l1, ref, rl, "VS sparse groups, head subset")
+    minf.minf_dense_attention(qc, kc, vc, scale=SCALE)  # unrelated work in between
+    o2, l2 = minf.minf_vs_attention(qc, kc, vc, vt, st, scale=SCALE, head_ids=ids)
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.uint8), o2.view(torch.uint8)) and torch.equal(l1, l2)
+
+
+def test_vs_only_sparse_groups_no_tiles(orc):
+    """Lone far offsets and no verticals: rows whose keys all come from the CUDA-core
+    pass (the tile kernel has nothing for them but offset 0's diagonal tile)."""
+    n = 1024
+    q, k, v = inputs(n, 1, 1, seed=44)
+    vi = np.full((1, 4), -1, np.int32)
+    si = np.array([[300, 700, 1000, -1]], np.int32)  # no offset 0: rows below 300 see no key
+    ref, rl = orc.vs_attention(q, k, v, SCALE, vi, si)
+    out, lse = minf.minf_vs_attention(*cuda(q, k, v), torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(),
+                                      scale=SCALE)
+    check_attention(out, lse, ref, rl, "VS lone offsets only")
+    assert torch.all(out[0, :300] == 0) and torch.all(torch.isneginf(lse[0, :300]))
