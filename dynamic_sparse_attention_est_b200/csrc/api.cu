@@ -23,7 +23,7 @@ thread_local std::string g_last_error;
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
 // Vertical-Slash routing of sparse slash groups to the CUDA-core pass: a tile
 // half is taken to cost this many offsets of that pass (0: tile kernel only).
-std::atomic<float> g_vs_diag_ratio{2.0f};
+std::atomic<float> g_vs_diag_ratio{1.0f};
 
 int fail(int code, const char *fmt, ...) {
     char buf[512];

@@ -11,17 +11,18 @@
 // takes those groups instead: for each query tile it stages the groups' key
 // ranges in 64-key chunks (K and V, by TMA, as the tile kernel does), and each
 // query row computes only its in-mask pairs, one dot product, one exponential
-// and one V update per offset, in fp32 with bf16 operands.
+// and one V update per offset (fp32 sums of products of bf16 operands).
 //
 // It produces a partial softmax state per query row over exactly those pairs
 // (each slash pair whose key is not a vertical key; verticals belong to the tile
 // kernel) -- the running max m and sum l in the log2 domain and the unnormalised
 // O -- which the tile kernel merges into its own in its epilogue.
 //
-// Roles (288 threads, one persistent CTA per SM striding over the work items):
-//   warps 0..7  consumers: two threads per query row (lane l of warp w holds row
-//               16 w + (l & 15) and head dims [64 (l >> 4), 64 (l >> 4) + 64))
-//   warp 8      TMA producer: one 64-key chunk of K and V per stage, 6 stages
+// Roles (384 threads, one persistent CTA per SM striding over the work items):
+//   warp 0      TMA producer: one 64-key chunk of K and V per stage, 6 stages
+//   warps 1..3  idle (they give their registers to the consumers and exit)
+//   warps 4..11 consumers: two threads per query row (lane l of warp 4 + w holds
+//               row 16 w + (l & 15) and head dims [64 (l >> 4), 64 (l >> 4) + 64))
 // A chunk stays until every consumer warp has moved past it; each warp releases
 // chunks in order, after it has seen them full.
 #include <algorithm>
@@ -35,23 +36,29 @@ namespace minf {
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kDiagThreads = (kConsumerWarps + 1) * 32;
+constexpr int kDiagThreads = 384;  // warpgroup 0: producer (warp 0) + 3 idle warps; warpgroups 1-2: consumers
+// Register split after setmaxnreg: the launch gives 384 threads x 168 registers (three
+// warps per SM sub-partition); warpgroup 0 drops to 40, the consumers rise to 232
+// (128 x 40 + 256 x 232 = 384 x 168).
+constexpr int kDiagRegsLaunch = 168;
+constexpr int kDiagRegsProducer = 40;
+constexpr int kDiagRegsConsumer = 232;
+static_assert(128 * kDiagRegsProducer + 256 * kDiagRegsConsumer <= kDiagThreads * kDiagRegsLaunch, "register split");
 constexpr int kDiagStages = 6;
 constexpr uint32_t kChunkBytes = 32768;  // 64 keys x 128 dims x 2 B, K then V
 constexpr uint32_t kDiagSmem = kDiagStages * kChunkBytes + 256 + 1024;  // + barriers + alignment slack
 
-// acc + lo(a) lo(b) + hi(a) hi(b): bf16 operands, fp32 products and sums (one
-// rounding per fused multiply-add, as an fp32 FMA of the widened operands).
-__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float acc) {
-    float r;
+// (acc0, acc1) += (lo(a) lo(b), hi(a) hi(b)): bf16 operands, fp32 products and
+// sums (one rounding per fused multiply-add, as an fp32 FMA of the widened
+// operands); two independent accumulators.
+__device__ __forceinline__ void dot2_bf16(uint32_t a, uint32_t b, float &acc0, float &acc1) {
     asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\t"
-        "mov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
-        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-        : "=f"(r)
-        : "r"(a), "r"(b), "f"(acc));
-    return r;
+        "mov.b32 {al, ah}, %2;\n\t"
+        "mov.b32 {bl, bh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, ah, bh, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(a), "r"(b));
 }
 
 // (o0, o1) += p * (lo(v), hi(v)) with p and v bf16, o fp32.
@@ -104,6 +111,9 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     const uint32_t ring = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDiagStages * kChunkBytes);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kDiagStages);
+    // per stage: bit u set iff key (chunk start + u) is a vertical key (written by the
+    // producer before it arrives on the stage's full barrier)
+    uint64_t *vmask = bars + 2 * kDiagStages + 1;
     auto full_bar = [&](int s) { return smem_u32(bars + s); };
     auto empty_bar = [&](int s) { return smem_u32(bars + kDiagStages + s); };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,7 +130,9 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     const WaitCtl wc{abort_flag, P.hdr ? &P.hdr->status : nullptr, P.wait_limit_ns};
     const int n_items = P.n_heads * P.n_qtiles;
 
-    if (warp == kConsumerWarps) {
+    if (warp < 4) {
+        setmaxnreg_dec<kDiagRegsProducer>();
+        if (warp != 0) return;
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&P.tmap_k);
@@ -135,6 +147,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
             const int ng = P.ngroups[hp];
             const int4 *groups = P.groups + (size_t)hp * P.gstride;
             const int g = P.head_ids[hp] / P.group;
+            const uint32_t *bv = P.bits_v + (size_t)hp * P.bit_stride;
             const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, P.n - 1);
             for (int gi = 0; ok && gi < ng; ++gi) {
                 const int4 G = __ldg(groups + gi);
@@ -143,13 +156,14 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                 const int nc = (b - a + kHalf) / kHalf;
                 for (int j = 0; j < nc; ++j, ++c) {
                     const int s = c % kDiagStages;
-                    const bool got = wait_bounded(empty_bar(s), ((c / kDiagStages) & 1) ^ 1, wc, wait_site(8, s, c));
+                    const bool got = wait_bounded_sleep(empty_bar(s), ((c / kDiagStages) & 1) ^ 1, wc, wait_site(8, s, c));
                     if (!__all_sync(0xffffffffu, got)) {
                         ok = false;
                         break;
                     }
                     tma_load_kv_chunk_warp(ring + s * kChunkBytes, &P.tmap_k, &P.tmap_v, full_bar(s), a + j * kHalf,
                                            g);
+                    if (lane == 0) vmask[s] = bits64_at(bv, P.n >> 5, a + j * kHalf);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full_bar(s));
                 }
@@ -166,11 +180,14 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     }
 
     // ---------------------------------------------------------------- consumers
-    const int rw = warp * 16;           // first row of this warp
+    setmaxnreg_inc<kDiagRegsConsumer>();
+    const int rw = (warp - 4) * 16;     // first row of this warp
     const int r = rw + (lane & 15);     // query row in the tile
     const int hf = lane >> 4;           // head-dimension half
     const float sl2 = P.scale_log2;
-    const uint32_t kbase = ring + hf * 8192, vbase = ring + 16384 + hf * 8192;
+    const uint32_t kbase = ring + hf * 8192;  // this thread's K box of a stage; its V box is 16 KB further
+    const uint32_t *vmask32 = reinterpret_cast<const uint32_t *>(vmask);
+    int win_lo = -1, st_lo = 0;  // first chunk of the current window and its stage
     int c_base = 0;  // sequence number of the current group's first chunk
     int got = 0;     // chunks [0, got) seen full by this warp
     int rel = 0;     // chunks [0, rel) released by this warp
@@ -178,7 +195,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     unsigned long long pairs = 0;
     auto see = [&]() -> bool {  // waits for chunk `got` to be full (warp-uniform)
         const int s = got % kDiagStages;
-        const bool gfull = wait_bounded(full_bar(s), (got / kDiagStages) & 1, wc, wait_site(9, s, got));
+        const bool gfull = wait_bounded_sleep(full_bar(s), (got / kDiagStages) & 1, wc, wait_site(9, s, got));
         if (!__all_sync(0xffffffffu, gfull)) return false;
         ++got;
         return true;
@@ -210,12 +227,11 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
         const int h = P.head_ids[hp];
         const int4 *groups = P.groups + (size_t)hp * P.gstride;
         const int *offs = P.offs + (size_t)hp * P.ostride;
-        const uint32_t *bv = P.bits_v + (size_t)hp * P.bit_stride;
         const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, P.n - 1);
         const int qi = r0 + r;
         const bool row_ok = qi <= rmax;
         const int last_r = rmax - r0;  // last valid row of the tile
-        uint32_t qv[32];
+        uint32_t qv[32];  // this thread's 64 query dims, bf16 pairs
         {
             const uint4 *src =
                 reinterpret_cast<const uint4 *>(P.q + ((size_t)h * P.n + min(qi, P.n - 1)) * kD + hf * 64);
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                 qv[4 * i + 3] = x.w;
             }
         }
-        float o[64];
+        float o[64];  // unnormalised O over this thread's 64 dims
 #pragma unroll
         for (int e = 0; e < 64; ++e) o[e] = 0.f;
         float m = -INFINITY, l = 0.f;
@@ -237,62 +253,72 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
             if (G.x > rmax) break;
             const int a = max(0, r0 - G.y), b = rmax - G.x;
             const int nc = (b - a + kHalf) / kHalf;
-            // offsets of the group from the largest down: the key ranges move forward
-            for (int j = G.w - 1; j >= 0; --j) {
-                const int off = __ldg(offs + G.z + j);
-                const int u0 = r0 - off - a;  // range position of row 0's key
-                const int ulo = max(0, u0 + rw), uhi = min(u0 + rw + 15, u0 + last_r);
-                if (ulo > uhi) continue;  // no valid row of this warp meets a key of this offset
-                if (!need(c_base + (ulo >> 6), c_base + (uhi >> 6))) {
-                    ok = false;
-                    break;
-                }
-                const int u = u0 + r;
-                bool use = row_ok && u >= 0;
-                if (use) {
-                    const int key = a + u;
-                    use = !((__ldg(bv + (key >> 5)) >> (key & 31)) & 1u);  // verticals are the tile kernel's
-                }
-                float s = 0.f;
-                uint32_t row_off = 0;
-                int sw = 0;
-                if (use) {
-                    const int ur = u & 63;
-                    row_off = (uint32_t)((c_base + (u >> 6)) % kDiagStages) * kChunkBytes + (uint32_t)ur * 128;
-                    sw = ur & 7;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint4 kk = lds128(kbase + row_off + ((i ^ sw) << 4));
-                        acc[0] = dot2_bf16(kk.x, qv[4 * i], acc[0]);
-                        acc[1] = dot2_bf16(kk.y, qv[4 * i + 1], acc[1]);
-                        acc[2] = dot2_bf16(kk.z, qv[4 * i + 2], acc[2]);
-                        acc[3] = dot2_bf16(kk.w, qv[4 * i + 3], acc[3]);
+            // offsets of the group from the largest down (the key ranges move forward),
+            // 32 at a time: lane l holds the l-th of the batch, broadcast by shuffle
+            for (int top = G.w - 1; ok && top >= 0; top -= 32) {
+                const int cnt = min(32, top + 1);
+                const int my_off = lane < cnt ? __ldg(offs + G.z + top - lane) : 0;
+                for (int jj = 0; jj < cnt; ++jj) {
+                    const int off = __shfl_sync(0xffffffffu, my_off, jj);
+                    const int u0 = r0 - off - a;  // range position of row 0's key
+                    const int ulo = max(0, u0 + rw), uhi = min(u0 + rw + 15, u0 + last_r);
+                    if (ulo > uhi) continue;  // no valid row of this warp meets a key of this offset
+                    const int clo = c_base + (ulo >> 6), chi = c_base + (uhi >> 6);
+                    if (clo != win_lo || chi >= got) {  // the window moved: release below it, see it full
+                        if (!need(clo, chi)) {
+                            ok = false;
+                            break;
+                        }
+                        win_lo = clo;
+                        st_lo = clo % kDiagStages;
                     }
-                    s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                }
-                s += __shfl_xor_sync(0xffffffffu, s, 16);  // the two halves of the row's dot product
-                if (use) {
-                    const float x = s * sl2;
-                    if (x > m + 8.0f) {  // the running max moves only when it grows by more than 2^8
-                        const float alpha = ex2_approx(m - x);  // 0 while m = -inf
+                    const int u = u0 + r;
+                    const bool in = row_ok && u >= 0;
+                    const int uc = max(u, 0);
+                    // the row's chunk is the window's first or second (the 16 rows span at most two)
+                    int st = st_lo + ((uc >> 6) - (ulo >> 6));
+                    if (st >= kDiagStages) st -= kDiagStages;
+                    const int ur = uc & 63;
+                    // in the mask unless the key is a vertical (those are the tile kernel's)
+                    const bool use = in && !((vmask32[2 * st + (ur >> 5)] >> (ur & 31)) & 1u);
+                    // row ur of the stage; its 16-byte chunk i sits at chunk i ^ (ur & 7) (128B swizzle)
+                    const uint32_t ka = kbase + (uint32_t)st * kChunkBytes + (uint32_t)ur * 128 + ((ur & 7) << 4);
+                    float s = 0.f;
+                    if (use) {
+                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight chains of 8
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) o[e] *= alpha;
-                        l *= alpha;
-                        m = x;
+                        for (int i = 0; i < 8; ++i) {
+                            const uint4 kk = lds128(ka ^ (i << 4));
+                            dot2_bf16(kk.x, qv[4 * i], acc[0], acc[1]);
+                            dot2_bf16(kk.y, qv[4 * i + 1], acc[2], acc[3]);
+                            dot2_bf16(kk.z, qv[4 * i + 2], acc[4], acc[5]);
+                            dot2_bf16(kk.w, qv[4 * i + 3], acc[6], acc[7]);
+                        }
+                        s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                     }
-                    const float p = ex2_approx(x - m);
-                    l += p;
-                    const uint16_t pb = bf16_bits(p);
+                    s += __shfl_xor_sync(0xffffffffu, s, 16);  // the two halves of the row's dot product
+                    if (use) {
+                        const float x = s * sl2;
+                        if (x > m + 8.0f) {  // the running max moves only when it grows by more than 2^8
+                            const float alpha = ex2_approx(m - x);  // 0 while m = -inf
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint4 vv = lds128(vbase + row_off + ((i ^ sw) << 4));
-                        axpy2_bf16(vv.x, pb, o[8 * i], o[8 * i + 1]);
-                        axpy2_bf16(vv.y, pb, o[8 * i + 2], o[8 * i + 3]);
-                        axpy2_bf16(vv.z, pb, o[8 * i + 4], o[8 * i + 5]);
-                        axpy2_bf16(vv.w, pb, o[8 * i + 6], o[8 * i + 7]);
+                            for (int e = 0; e < 64; ++e) o[e] *= alpha;
+                            l *= alpha;
+                            m = x;
+                        }
+                        const float p = ex2_approx(x - m);
+                        l += p;
+                        const uint16_t pb = bf16_bits(p);  // P enters P V in bf16, as on the tensor cores
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint4 vvi = lds128((ka + 16384) ^ (i << 4));
+                            axpy2_bf16(vvi.x, pb, o[8 * i], o[8 * i + 1]);
+                            axpy2_bf16(vvi.y, pb, o[8 * i + 2], o[8 * i + 3]);
+                            axpy2_bf16(vvi.z, pb, o[8 * i + 4], o[8 * i + 5]);
+                            axpy2_bf16(vvi.w, pb, o[8 * i + 6], o[8 * i + 7]);
+                        }
+                        ++pairs;  // counted by both threads of the row, halved at the end
                     }
-                    pairs += hf == 0;
                 }
             }
             if (!ok) break;
@@ -317,6 +343,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     if (P.hdr) {
 #pragma unroll
         for (int sft = 16; sft > 0; sft >>= 1) pairs += __shfl_xor_sync(0xffffffffu, pairs, sft);
+        pairs >>= 1;  // both threads of each row counted its pairs
         if (lane == 0 && pairs) {
             atomicAdd(&P.hdr->pairs, pairs);
             atomicAdd(&P.hdr->diag_pairs, pairs);
@@ -329,6 +356,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
 cudaError_t run_vs_diag(const DiagParams &P, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(vs_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
     if (e != cudaSuccess) return e;
+    // setmaxnreg.inc waits for registers the launch reserved: refuse to launch a
+    // build whose register count at entry would make the split wait forever
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, vs_diag_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kDiagRegsLaunch) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -36,6 +36,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: a thread whose phase is not yet complete may
+// be suspended for up to `ns` nanoseconds, woken early when the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -78,6 +91,21 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (*w.abort_flag) return false;
+        if (globaltimer_ns() - t0 > w.limit_ns) {
+            wait_gave_up(w, site);
+            return false;
+        }
+    }
+}
+
+// wait_bounded with suspended waiting (see mbar_try_wait_hint): far fewer
+// instructions issued while a warp waits, for kernels whose waits are long.
+__device__ __forceinline__ bool wait_bounded_sleep(uint32_t bar, uint32_t parity, const WaitCtl &w, int site = 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (*w.abort_flag) return false;
         if (globaltimer_ns() - t0 > w.limit_ns) {
             wait_gave_up(w, site);

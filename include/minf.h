@@ -278,7 +278,9 @@ void minf_set_wait_limit_ns(uint64_t ns);
  * per offset) when m < ratio * H.  The result is the same token-exact masked
  * softmax either way (the two partial states are merged per row); only the
  * time differs.  ratio <= 0 sends every group to the tensor cores.  Default
- * 2.0; applies to minf_vs_attention and the mixed layer (not to
+ * 1.0 (on B200 a lone offset costs the CUDA-core pass about as much as two
+ * thirds of a 128x128 tensor-core tile, a triple about as much as its four
+ * half-tiles); applies to minf_vs_attention and the mixed layer (not to
  * minf_vs_attention_tiles), process-wide, for calls made after it.
  */
 void minf_set_vs_diag_ratio(float ratio);
