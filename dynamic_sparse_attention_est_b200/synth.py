@@ -70,6 +70,10 @@ WORKLOADS: Dict[str, Workload] = {
                                  n_sink=128, window=4096),
     "trishape-gqa-128k": Workload("trishape-gqa-128k", "trishape", 32, 8, 131072, "plain",
                                    n_sink=128, window=4096, last_q=64),
+    # one Vertical-Slash head at 256K tokens with the layer's budgets: a profiling-size case
+    # for the sparse-slash pass (a few hundred MB on the device)
+    "vs-1h-256k": Workload("vs-1h-256k", "vs", 1, 1, 262144, "vertical", heavy_frac=0.005,
+                            last_q=64, n_vertical=1000, n_slash=6096),
     # one Vertical-Slash head at 1M tokens with the layer's budgets: a profiling-size case
     "vs-1h-1m": Workload("vs-1h-1m", "vs", 1, 1, 1048576, "vertical", heavy_frac=0.005,
                           last_q=64, n_vertical=1000, n_slash=6096),
