@@ -57,6 +57,9 @@ struct Carver {
 
 int qtiles(int n) { return (n + kTileM - 1) / kTileM; }
 
+// Vertical-Slash tile kernel launch order: kv-head-major from this length on.
+constexpr int kVsKvMajorFrom = 1 << 18;
+
 // Vertical-Slash estimate: key chunking for one wave of one CTA per SM (148 SMs;
 // the kernel's shared memory allows one CTA per SM), whole chunks per head pair.
 void vs_est_geometry(int n, int n_pairs, int *n_chunks, int *chunk_tiles, int *n_ktiles) {
@@ -365,7 +368,10 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
     if (e != cudaSuccess) return cuda_fail(e, "vs plan launch");
     AttnParams P;
     memset(&P, 0, sizeof(P));
-    fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
+    // long sequences launch kv-head-major (one kv-head's q-heads side by side), so that
+    // the CTAs in flight share that kv-head's K and V in L2 (at 32K heads side by side
+    // measured faster)
+    fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id, c.n >= kVsKvMajorFrom);
     e = encode_attn_maps(P, q, k, v, c);
     if (e != cudaSuccess) return cuda_fail(e, "tensor map");
     if (ratio > 0.f) {
