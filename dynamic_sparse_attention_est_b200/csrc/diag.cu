@@ -26,6 +26,7 @@
 // A chunk stays until every consumer warp has moved past it; each warp releases
 // chunks in order, after it has seen them full.
 #include <algorithm>
+#include <climits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -149,10 +150,16 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
             const int g = P.head_ids[hp] / P.group;
             const uint32_t *bv = P.bits_v + (size_t)hp * P.bit_stride;
             const int r0 = t * kTileM, rmax = min(r0 + kTileM - 1, P.n - 1);
+            int2 gwin = make_int2(0, 0);
             for (int gi = 0; ok && gi < ng; ++gi) {
-                const int4 G = __ldg(groups + gi);
-                if (G.x > rmax) break;  // groups ascend: no row of this tile reaches the rest
-                const int a = max(0, r0 - G.y), b = rmax - G.x;
+                // first and last offsets of 32 groups at a time, broadcast by shuffle
+                if ((gi & 31) == 0) {
+                    const int4 w = gi + lane < ng ? __ldg(groups + gi + lane) : make_int4(INT_MAX, 0, 0, 0);
+                    gwin = make_int2(w.x, w.y);
+                }
+                const int gx = __shfl_sync(0xffffffffu, gwin.x, gi & 31), gy = __shfl_sync(0xffffffffu, gwin.y, gi & 31);
+                if (gx > rmax) break;  // groups ascend: no row of this tile reaches the rest
+                const int a = max(0, r0 - gy), b = rmax - gx;
                 const int nc = (b - a + kHalf) / kHalf;
                 for (int j = 0; j < nc; ++j, ++c) {
                     const int s = c % kDiagStages;
@@ -248,16 +255,25 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 64; ++e) o[e] = 0.f;
         float m = -INFINITY, l = 0.f;
+        // group descriptors 32 at a time: lane l holds group gw + l, broadcast by shuffle,
+        // so that no group waits on a load of its own descriptor
+        int4 gwin = make_int4(0, 0, 0, 0);
         for (int gi = 0; ok && gi < ng; ++gi) {
-            const int4 G = __ldg(groups + gi);
+            if ((gi & 31) == 0) gwin = gi + lane < ng ? __ldg(groups + gi + lane) : make_int4(INT_MAX, 0, 0, 0);
+            int4 G;
+            G.x = __shfl_sync(0xffffffffu, gwin.x, gi & 31);
+            G.y = __shfl_sync(0xffffffffu, gwin.y, gi & 31);
+            G.z = __shfl_sync(0xffffffffu, gwin.z, gi & 31);
+            G.w = __shfl_sync(0xffffffffu, gwin.w, gi & 31);
             if (G.x > rmax) break;
             const int a = max(0, r0 - G.y), b = rmax - G.x;
             const int nc = (b - a + kHalf) / kHalf;
             // offsets of the group from the largest down (the key ranges move forward),
-            // 32 at a time: lane l holds the l-th of the batch, broadcast by shuffle
+            // 32 at a time: lane l holds the l-th of the batch, broadcast by shuffle (a
+            // lone offset is the descriptor's own first offset: nothing to load)
             for (int top = G.w - 1; ok && top >= 0; top -= 32) {
                 const int cnt = min(32, top + 1);
-                const int my_off = lane < cnt ? __ldg(offs + G.z + top - lane) : 0;
+                const int my_off = G.w == 1 ? G.x : (lane < cnt ? __ldg(offs + G.z + top - lane) : 0);
                 for (int jj = 0; jj < cnt; ++jj) {
                     const int off = __shfl_sync(0xffffffffu, my_off, jj);
                     const int u0 = r0 - off - a;  // range position of row 0's key
@@ -297,15 +313,18 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                         s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                     }
                     s += __shfl_xor_sync(0xffffffffu, s, 16);  // the two halves of the row's dot product
-                    if (use) {
-                        const float x = s * sl2;
-                        if (x > m + 8.0f) {  // the running max moves only when it grows by more than 2^8
-                            const float alpha = ex2_approx(m - x);  // 0 while m = -inf
+                    const float x = s * sl2;
+                    // the running max moves only when it grows by more than 2^8; the rescale
+                    // of O is a branch the whole warp takes or skips together
+                    const bool grow = use && x > m + 8.0f;
+                    if (__any_sync(0xffffffffu, grow)) {
+                        const float alpha = grow ? ex2_approx(m - x) : 1.f;  // 0 while m = -inf
 #pragma unroll
-                            for (int e = 0; e < 64; ++e) o[e] *= alpha;
-                            l *= alpha;
-                            m = x;
-                        }
+                        for (int e = 0; e < 64; ++e) o[e] *= alpha;
+                        l *= alpha;
+                        m = grow ? x : m;
+                    }
+                    if (use) {
                         const float p = ex2_approx(x - m);
                         l += p;
                         const uint16_t pb = bf16_bits(p);  // P enters P V in bf16, as on the tensor cores
