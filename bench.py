@@ -347,8 +347,8 @@ def estimate_bytes(w) -> float:
     kv-head (256 B per key), the vertical and slash score rows are written once
     and read by five radix passes, the 191-offset diagonal partials are written
     and read once.  Block-Sparse: Q and K are read once for pooling, the pooled
-    rows written, and the lower triangle of pooled scores written once and read
-    once by the per-row selection.
+    rows written as three bf16 parts (768 B per block), and the lower triangle
+    of pooled scores written once and read once by the per-row selection.
     """
     n, hq, hkv = w.n, w.hq, w.hkv
     if w.pattern == "vs":
@@ -359,7 +359,7 @@ def estimate_bytes(w) -> float:
         return float(k_stream + scores + diag + hq * 64 * 256)
     if w.pattern == "block":
         nb = n // 64
-        pool = (hq + hkv) * n * 256 + (hq + hkv) * nb * 512
+        pool = (hq + hkv) * n * 256 + (hq + hkv) * nb * 768
         tri = hq * nb * (nb + 1) / 2 * 4
         return float(pool + 2 * tri)
     return 0.0

@@ -126,8 +126,8 @@ BsEstBufs carve_bs_est(Carver &c, int hkv, int n, int n_heads) {
     BsEstBufs b{};
     const size_t nb = (size_t)n / kBlock;
     b.head_batch = bs_head_batch(n, n_heads);
-    b.qp = c.take<float>((size_t)n_heads * nb * kD);
-    b.kp = c.take<float>((size_t)hkv * nb * kD);
+    b.qs = c.take<__nv_bfloat16>((size_t)n_heads * 3 * nb * kD);
+    b.ks = c.take<__nv_bfloat16>((size_t)hkv * 3 * nb * kD);
     b.scores = c.take<float>((size_t)b.head_batch * nb * nb);
     return b;
 }
@@ -421,7 +421,7 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
 }
 
 int do_block_estimate(const Common &c, const void *q, const void *k, int topk, int32_t *blk_idx, int32_t *blk_cnt,
-                      char *scratch, cudaStream_t st) {
+                      float *scores_out, void *ws, char *scratch, cudaStream_t st) {
     Carver cv(scratch, 0);
     BsEstBufs b = carve_bs_est(cv, c.hkv, c.n, c.n_heads);
     BsEstArgs a{};
@@ -435,6 +435,9 @@ int do_block_estimate(const Common &c, const void *q, const void *k, int topk, i
     a.head_ids = c.ids;
     a.blk_idx = blk_idx;
     a.blk_cnt = blk_cnt;
+    a.scores_out = scores_out;
+    a.hdr = ws;
+    a.wait_limit_ns = g_wait_limit_ns.load();
     cudaError_t e = run_block_estimate(a, b, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "block_estimate launch");
 }
@@ -646,7 +649,22 @@ int minf_block_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv,
     if (n / kBlock > 32768) return fail(MINF_ERR_UNSUPPORTED, "more than 32768 blocks");
     if ((rc = check_ws(ws, ws_bytes, bytes_bs_est(hkv, n, c.n_heads)))) return rc;
     if ((rc = select_device(q))) return rc;
-    return do_block_estimate(c, q, k, topk, blk_idx, blk_cnt, static_cast<char *>(ws) + MINF_STATUS_BYTES,
+    return do_block_estimate(c, q, k, topk, blk_idx, blk_cnt, nullptr, ws,
+                             static_cast<char *>(ws) + MINF_STATUS_BYTES, (cudaStream_t)stream);
+}
+
+int minf_block_scores(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d, int block,
+                      const int32_t *head_ids, int n_heads, float *scores, void *ws, size_t ws_bytes,
+                      minf_stream_t stream) {
+    Common c;
+    int rc = check_common(q, k, hq, hkv, n, d, head_ids, n_heads, c);
+    if (rc) return rc;
+    if (block != kBlock) return fail(MINF_ERR_UNSUPPORTED, "block %d (only 64)", block);
+    if (!scores) return fail(MINF_ERR_INVALID, "null scores");
+    if (n / kBlock > 32768) return fail(MINF_ERR_UNSUPPORTED, "more than 32768 blocks");
+    if ((rc = check_ws(ws, ws_bytes, bytes_bs_est(hkv, n, c.n_heads)))) return rc;
+    if ((rc = select_device(q))) return rc;
+    return do_block_estimate(c, q, k, 1, nullptr, nullptr, scores, ws, static_cast<char *>(ws) + MINF_STATUS_BYTES,
                              (cudaStream_t)stream);
 }
 
@@ -786,7 +804,7 @@ int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v,
                                  scratch_vs, true, st);
     }
     if (sub[PAT_BLOCK].n_heads) {
-        rc2 = do_block_estimate(sub[PAT_BLOCK], q, k, topk, blk_idx, blk_cnt, scratch_bs, st2);
+        rc2 = do_block_estimate(sub[PAT_BLOCK], q, k, topk, blk_idx, blk_cnt, nullptr, ws, scratch_bs, st2);
         if (!rc2)
             rc2 = do_block_attention(sub[PAT_BLOCK], q, k, v, scale, blk_idx, blk_cnt, topk, out, lse, ws,
                                      scratch_bs, true, st2);

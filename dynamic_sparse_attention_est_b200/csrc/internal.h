@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -84,9 +85,9 @@ cudaError_t run_vs_estimate(const VsEstArgs &a, const VsEstBufs &b, cudaStream_t
 
 // Block-Sparse estimation.
 struct BsEstBufs {
-    float *qp;       // [n_heads][nb][128]
-    float *kp;       // [hkv][nb][128]
-    float *scores;   // [head_batch][nb][nb]
+    __nv_bfloat16 *qs;  // [n_heads][3][nb][128] pooled Q as hi, mid, lo bf16 parts
+    __nv_bfloat16 *ks;  // [hkv][3][nb][128]
+    float *scores;      // [head_batch][nb][nb]
     int head_batch;
 };
 
@@ -95,6 +96,9 @@ struct BsEstArgs {
     int hq, hkv, n, n_heads, topk;
     const int *head_ids;  // host
     int *blk_idx, *blk_cnt;
+    float *scores_out;    // when set: the pooled scores of every listed head go here, no selection
+    void *hdr;            // WsHeader*
+    unsigned long long wait_limit_ns;
 };
 
 cudaError_t run_block_estimate(const BsEstArgs &a, const BsEstBufs &b, cudaStream_t st);

@@ -48,6 +48,7 @@ _SIGS = {
                                    _P]),
     "minf_vs_attention_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_block_estimate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "minf_block_scores": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "minf_block_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "minf_ashape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "minf_trishape_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -253,6 +254,20 @@ def minf_block_estimate(q, k, topk: int = 100, block: int = 64, head_ids=None, w
                                      _ptr(blk_cnt), _ptr(ws), ws.numel(), _stream(q.device)),
            "minf_block_estimate")
     return blk_idx, blk_cnt
+
+
+def minf_block_scores(q, k, block: int = 64, head_ids=None, ws=None):
+    """Pooled block scores [n_heads][n/64][n/64] (fp32); entries j > i unspecified."""
+    hq, hkv, n, d = _qkv(q, k)
+    ids, nh = _heads(hq, head_ids)
+    need = workspace_bytes(OP_BLOCK_ESTIMATE, hq, hkv, n, nh, 1)
+    ws = _ws_for(ws, need, q.device)
+    nb = n // 64
+    scores = torch.empty(nh, nb, nb, dtype=torch.float32, device=q.device)
+    _check(lib().minf_block_scores(_ptr(q), _ptr(k), hq, hkv, n, d, block, ids, nh, _ptr(scores), _ptr(ws),
+                                   ws.numel(), _stream(q.device)),
+           "minf_block_scores")
+    return scores
 
 
 def minf_block_attention(q, k, v, blk_idx, blk_cnt, scale: Optional[float] = None, head_ids=None, out=None,

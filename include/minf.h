@@ -168,11 +168,31 @@ int minf_vs_attention_tiles(const minf_bf16 *q, const minf_bf16 *k, const minf_b
  * kept; the best topk-1 blocks j < i join it (ties to the lower j).  Output,
  * ASCENDING, -1 padded:
  *   blk_idx int32 [n_heads][n/64][topk], blk_cnt int32 [n_heads][n/64].
+ * The scores are computed on the tensor cores from three bf16 parts of each
+ * pooled fp32 value (the part products down to 2^-16 relative size, fp32
+ * accumulation): their error stays below that of an fp32 dot product.  A
+ * bounded wait that gives up records MINF_ERR_TIMEOUT in the workspace's
+ * status block (minf_status).
  */
 int minf_block_estimate(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
                         int block, int topk, const int32_t *head_ids, int n_heads,
                         int32_t *blk_idx, int32_t *blk_cnt, void *ws, size_t ws_bytes,
                         minf_stream_t stream);
+
+/*
+ * The pooled block scores behind minf_block_estimate, for inspection and for
+ * callers with their own selection ([NEWS] 方法介绍: the pooled product
+ * estimates the block means of the attention logits).  Writes, for each
+ * listed head p, query block i and key block j <= i,
+ *   scores[p][i][j] = Qp_i . Kp_j          (fp32, device, [n_heads][n/64][n/64])
+ * with the same arithmetic as minf_block_estimate; entries j > i are
+ * unspecified (some are written).  The caller owns `scores`; workspace as
+ * MINF_OP_BLOCK_ESTIMATE (its score rows stay unused).  Errors as
+ * minf_block_estimate; a null `scores` is MINF_ERR_INVALID.
+ */
+int minf_block_scores(const minf_bf16 *q, const minf_bf16 *k, int hq, int hkv, int n, int d,
+                      int block, const int32_t *head_ids, int n_heads, float *scores, void *ws,
+                      size_t ws_bytes, minf_stream_t stream);
 
 /*
  * Block-Sparse attention: query i of head position p attends to key k iff

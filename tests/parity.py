@@ -37,11 +37,30 @@ def _gamma(m):
 # |p| <= a and |p^| <= (1 + gamma_63) a:
 #   |s^ - s| <= [gamma_128 (1 + gamma_63)^2 + 2 gamma_63 + gamma_63^2] sum_d a_d b_d.
 BS_ERR_COEF = _gamma(128) * (1 + _gamma(63)) ** 2 + 2 * _gamma(63) + _gamma(63) ** 2
+# That bound is the index band's floor.  The GPU's own score arithmetic stays
+# inside a smaller one.  It keeps each pooled fp32 value p^ as three bf16 parts
+# h + m + l with |p^ - h - m - l| <= 2^-24 |p^| (three roundings to 8 significant
+# bits; each residual is exact in fp32).  Of the nine part products it forms the
+# six down to 2^-16 relative size, dropping (with the residuals) at most
+# (4 + 2^-6) 2^-24 |p^q||p^k| per term; bf16 products are exact in fp32.  The
+# tensor core's fp32 accumulation is modelled as: one K = 16 step returns
+# c + (its 16 products) within 2^-22 (|c| + sum |p|), i.e. within two fp32 ulps
+# (truncation and a lost guard bit).  The five small part products, together
+# at most BS_TC_SMALL of S = sum |p^q||p^k|, take the first 40 steps (each step
+# with |c| + sum |p| <= 2 BS_TC_SMALL S); the eight hi.hi steps follow, each
+# with |c| + sum |p| <= (BS_TC_SMALL + (1 + 2^-8)^2) S.
+BS_TC_SMALL = (2 * 2.0 ** -8 + 3 * 2.0 ** -16) * (1 + 2.0 ** -8) ** 2
+BS_TC_STEP = 2.0 ** -22
+# the accumulation alone, per unit of S (the pooled values' sum_d |p^q||p^k|)
+BS_TC_ACC_COEF = BS_TC_STEP * (40 * 2 * BS_TC_SMALL + 8 * (BS_TC_SMALL + (1 + 2.0 ** -8) ** 2))
+BS_TC_ERR_COEF = ((4 + 2.0 ** -6) * U32 + BS_TC_ACC_COEF) * (1 + _gamma(63)) ** 2 \
+    + 2 * _gamma(63) + _gamma(63) ** 2
 
 
-def bs_score_error(q, k, block=64):
-    """Per (q-head, query block i): twice the largest worst-case fp32 error of the
-    GPU's pooled scores s_ij over the candidates j < i (zero for i = 0).
+def bs_score_error(q, k, block=64, coef=BS_ERR_COEF):
+    """Per (q-head, query block i): twice the largest worst-case error (coef per
+    unit of sum_d a b; the fp32 dot-product bound by default) of the pooled
+    scores s_ij over the candidates j < i (zero for i = 0).
 
     With that error at most E on every candidate of a row, an item whose exact
     score exceeds the k-th best exact score t by more than 2E outranks, on the GPU,
@@ -59,8 +78,71 @@ def bs_score_error(q, k, block=64):
     below = np.tril(np.ones((nb, nb), bool), -1)
     for h in range(hq):
         m = aq[h] @ ak[h // (hq // hkv)].T
-        out[h] = 2.0 * BS_ERR_COEF * np.where(below, m, 0.0).max(axis=1)
+        out[h] = 2.0 * coef * np.where(below, m, 0.0).max(axis=1)
     return out
+
+
+def bs_score_bound(q, k, block=64, coef=BS_TC_ERR_COEF):
+    """Per (q-head, i, j): coef * sum_d a_i,d b_j,d, the worst-case error of one
+    pooled score (a, b the block means of |q| and |k|)."""
+    qa = np.abs(to_np(q))
+    ka = np.abs(to_np(k))
+    hq, n, d = qa.shape
+    hkv = ka.shape[0]
+    nb = n // block
+    aq = qa.reshape(hq, nb, block, d).mean(axis=2)
+    ak = ka.reshape(hkv, nb, block, d).mean(axis=2)
+    g = hq // hkv
+    return coef * np.stack([aq[h] @ ak[h // g].T for h in range(hq)])
+
+
+def pooled_fp32_model(x):
+    """Block means as the GPU forms them: sequential fp32 sums of 64 rows, times 1/64."""
+    x = x.float().numpy()
+    h, n, d = x.shape
+    xb = x.reshape(h, n // 64, 64, d)
+    acc = np.zeros((h, n // 64, d), np.float32)
+    for r in range(64):
+        acc = (acc + xb[:, :, r, :]).astype(np.float32)
+    return (acc * np.float32(1.0 / 64)).astype(np.float32)
+
+
+def _bf16_parts(p):
+    """hi, mid, lo bf16 parts of fp32 values (round to nearest even at each step)."""
+    parts, r = [], torch.from_numpy(p)
+    for _ in range(3):
+        b = r.to(torch.bfloat16).float()
+        parts.append(b.numpy().astype(np.float64))
+        r = (r - b).float()  # exact in fp32
+    return parts
+
+
+def _trunc_f32(x):
+    """fp64 -> fp32 rounded toward zero."""
+    f = x.astype(np.float32)
+    over = np.abs(f.astype(np.float64)) > np.abs(x)
+    f[over] = np.nextafter(f[over], np.float32(0))
+    return f
+
+
+def tc_pooled_scores_model(q, k, products=("hl", "mm", "hm", "lh", "mh", "hh")):
+    """Emulation of the tensor-core score arithmetic: split parts, the listed
+    part products (Q part, K part) in order, each 128-deep product as eight
+    K = 16 steps whose 16 exact products and the accumulator are summed exactly
+    and truncated to fp32 (a pessimistic accumulation)."""
+    qp, kp = pooled_fp32_model(q), pooled_fp32_model(k)
+    qs, ks = _bf16_parts(qp), _bf16_parts(kp)
+    idx = {"h": 0, "m": 1, "l": 2}
+    g = q.shape[0] // k.shape[0]
+    out = []
+    for h in range(q.shape[0]):
+        c = np.zeros((qp.shape[1], kp.shape[1]), np.float32)
+        for pr in products:
+            a, b = qs[idx[pr[0]]][h], ks[idx[pr[1]]][h // g]
+            for s0 in range(0, 128, 16):
+                c = _trunc_f32(c.astype(np.float64) + a[:, s0:s0 + 16] @ b[:, s0:s0 + 16].T)
+        out.append(c.astype(np.float64))
+    return np.stack(out)
 
 
 def to_np(t):

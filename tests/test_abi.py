@@ -98,6 +98,10 @@ def test_estimate_argument_checks(minf_lib):
                                  None) == minf.MINF_ERR_UNSUPPORTED
     assert L.minf_block_estimate(FAKE, FAKE, 4, 2, 1024, 128, 64, 0, None, 4, FAKE, FAKE, FAKE, 1 << 30,
                                  None) == minf.MINF_ERR_INVALID
+    assert L.minf_block_scores(FAKE, FAKE, 4, 2, 1024, 128, 32, None, 4, FAKE, FAKE, 1 << 30,
+                               None) == minf.MINF_ERR_UNSUPPORTED
+    assert L.minf_block_scores(FAKE, FAKE, 4, 2, 1024, 128, 64, None, 4, None, FAKE, 1 << 30,
+                               None) == minf.MINF_ERR_INVALID
     assert L.minf_ashape_attention(FAKE, FAKE, FAKE, 4, 2, 1024, 128, 0.1, None, 4, -1, 10, FAKE, None, FAKE,
                                    256, None) == minf.MINF_ERR_INVALID
     codes = (ctypes.c_int8 * 4)(1, 2, 3, 7)

@@ -10,7 +10,8 @@ import pytest
 import torch
 
 from dynamic_sparse_attention_est_b200 import minf, synth
-from parity import bs_score_error, check_attention, check_topk_band, check_topp, to_np
+from parity import (BS_TC_ACC_COEF, bs_score_bound, bs_score_error, check_attention, check_topk_band, check_topp,
+                    pooled_fp32_model, tc_pooled_scores_model, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -82,6 +83,38 @@ def test_block_estimate_band(orc, n, hq, hkv, topk):
             assert row[-1] == i, "diagonal block forced"
             check_topk_band(row[:-1], sc[hp, i, :i], topk - 1, f"block row {hp}/{i}", abs_band=eb[hp, i])
             assert np.all(gi[hp, i, gc[hp, i]:] == -1)
+
+
+@pytest.mark.parametrize("n,hq,hkv,ids", [(64 * 300, 4, 2, [3, 0, 2]),   # three row tiles, the last ragged
+                                           (64 * 263, 2, 1, None),        # nb % 4 != 0: scalar stores
+                                           (64 * 5, 2, 2, None)])         # one tile, fewer rows than a TMA box
+def test_block_scores_tensor_core_error(orc, n, hq, hkv, ids):
+    """The tensor-core pooled scores, entry by entry for j <= i:
+    - against the exact (fp64) scores, within the worst-case bound of the split-bf16
+      arithmetic (which lies inside the fp32 dot-product bound of the index band);
+    - against a CPU model of the same arithmetic (identical fp32 pooling and bf16
+      parts, truncating fp32 accumulation per K = 16 step), within twice the bound
+      of the accumulation alone: a missing or misplaced part product fails this."""
+    w = synth.Workload("t", "block", hq, hkv, n, "clustered")
+    x = synth.generate(w, seed=4)
+    q, k = x["q"], x["k"]
+    heads = list(range(hq)) if ids is None else ids
+    _, _, _, _, sc = orc.block_estimate(q, k, 64, 1, head_ids=heads, return_scores=True)
+    gs = minf.minf_block_scores(*cuda(q, k), head_ids=ids).cpu().numpy().astype(np.float64)
+    nb = n // 64
+    tril = np.tril(np.ones((nb, nb), bool))
+    bound = bs_score_bound(q, k)[heads]
+    model = tc_pooled_scores_model(q, k)[heads]
+    qp, kp = np.abs(pooled_fp32_model(q).astype(np.float64)), np.abs(pooled_fp32_model(k).astype(np.float64))
+    g = hq // hkv
+    s_abs = np.stack([qp[h] @ kp[h // g].T for h in heads])
+    for hp in range(len(heads)):
+        err = np.abs(gs[hp] - sc[hp])[tril]
+        assert np.all(np.isfinite(gs[hp][tril]))
+        assert np.all(err <= bound[hp][tril]), f"head {heads[hp]}: max err/bound {np.max(err / bound[hp][tril]):.3g}"
+        dm = np.abs(gs[hp] - model[hp])[tril]
+        lim = 2 * BS_TC_ACC_COEF * s_abs[hp][tril]
+        assert np.all(dm <= lim), f"head {heads[hp]}: max |gpu - model| / limit {np.max(dm / lim):.3g}"
 
 
 def _rand_vs_indices(rng, n, nh, nv, ns):
@@ -584,3 +617,37 @@ def test_vs_only_sparse_groups_no_tiles(orc):
                                       scale=SCALE)
     check_attention(out, lse, ref, rl, "VS lone offsets only")
     assert torch.all(out[0, :300] == 0) and torch.all(torch.isneginf(lse[0, :300]))
+
+
+# ----------------------------------------------------------------------------- counters and launch timing
+def test_stats_detail_and_launch_timing():
+    """Per-kernel counters add up to the totals and match the dense tile count; the
+    launch timing names every kernel sequence of the call, once per call."""
+    n, hq, hkv = 1088, 2, 1
+    q, k, v = cuda(*inputs(n, hq, hkv, seed=2))
+    ws = minf.workspace(256, q.device)
+    minf.minf_profile_read()  # nothing pending
+    minf.minf_profile_enable(True)
+    try:
+        minf.minf_dense_attention(q, k, v, scale=SCALE, ws=ws)
+        minf.minf_dense_attention(q, k, v, scale=SCALE, ws=ws)
+    finally:
+        minf.minf_profile_enable(False)
+    prof = minf.minf_profile_read()
+    assert set(prof) == {"attn_kernel<DENSE>"} and prof["attn_kernel<DENSE>"][0] == 2
+    assert prof["attn_kernel<DENSE>"][1] > 0
+    assert minf.minf_profile_read() == {}  # read clears
+    det = minf.minf_stats_detail(ws)
+    nt = (n + 127) // 128
+    dense_tiles = hq * sum((min(2 * t + 2, n // 64) + 1) // 2 for t in range(nt))
+    assert det["tiles"] == det["tiles_dense"] == dense_tiles
+    assert det["tiles_vs"] == det["tiles_block"] == det["tiles_ashape"] == det["diag_pairs"] == 0
+    assert det["pairs"] == hq * n * (n + 1) // 2
+    # Vertical-Slash with lone offsets: the CUDA-core pass's pairs are part of the total
+    vi = np.full((hq, 4), -1, np.int32)
+    si = np.array([[0, 300, 700, -1], [5, 500, -1, -1]], np.int32)
+    wsv = minf.workspace(minf.workspace_bytes(minf.OP_VS_ATTENTION, hq, hkv, n, hq, 4, 4), q.device)
+    minf.minf_vs_attention(q, k, v, torch.from_numpy(vi).cuda(), torch.from_numpy(si).cuda(), scale=SCALE, ws=wsv)
+    det = minf.minf_stats_detail(wsv)
+    assert det["pairs"] == sum(n - o for o in (0, 300, 700, 5, 500))
+    assert 0 < det["diag_pairs"] <= det["pairs"] and det["tiles"] == det["tiles_vs"]

@@ -1,19 +1,22 @@
-"""The comparison rules themselves, on the CPU: the index tie band and the
-Block-Sparse fp32 error floor that widens it.
+"""The comparison rules themselves, on the CPU: the index tie band, the
+Block-Sparse fp32 error floor that widens it, and the error model of the
+tensor-core pooled scores.
 """
 import numpy as np
 import torch
 
 from dynamic_sparse_attention_est_b200 import synth
-from parity import BS_ERR_COEF, bs_score_error, check_topk_band
+from parity import (BS_ERR_COEF, BS_TC_ERR_COEF, bs_score_bound, bs_score_error,
+                    check_topk_band, tc_pooled_scores_model)
 
 import pytest
 
 
-def _gpu_like_pooled_scores(q, k):
-    """fp32 emulation of the GPU's Block-Sparse score arithmetic: sequential fp32
-    sums of the 64 rows of a block, times 1/64, then 128 sequential fp32 FMAs
-    (each FMA emulated as an exact fp64 product-sum rounded once to fp32)."""
+def _fp32_pooled_scores(q, k):
+    """fp32 emulation of an fp32 pooled-score dot product (the arithmetic the
+    index band's floor is derived for): sequential fp32 sums of the 64 rows of a
+    block, times 1/64, then 128 sequential fp32 FMAs (each FMA emulated as an
+    exact fp64 product-sum rounded once to fp32)."""
     q = q.float().numpy()
     k = k.float().numpy()
     hq, n, d = q.shape
@@ -47,7 +50,7 @@ def test_bs_error_floor_bounds_fp32_pooled_scores(structure):
     nb = q.shape[1] // 64
     exact = np.einsum("hid,hjd->hij", q.double().numpy().reshape(2, nb, 64, 128).mean(2),
                       k.double().numpy().reshape(1, nb, 64, 128).mean(2).repeat(2, 0))
-    got = _gpu_like_pooled_scores(q, k).astype(np.float64)
+    got = _fp32_pooled_scores(q, k).astype(np.float64)
     eb = bs_score_error(q, k)  # twice the per-row bound
     err = np.abs(got - exact)
     for h in range(2):
@@ -92,3 +95,21 @@ def test_band_floor_admits_near_zero_ties():
     check_topk_band(np.array([0, 1, 3]), s, 3, "with floor", abs_band=1e-6)
     with pytest.raises(AssertionError):
         check_topk_band(np.array([0, 1, 4]), s, 3, "clear loser", abs_band=1e-6)
+
+
+@pytest.mark.parametrize("structure", ["clustered", "plain"])
+def test_tensor_core_score_model_within_its_bound(structure):
+    w = synth.Workload("t", "block", 2, 1, 64 * 40, structure)
+    x = synth.generate(w, seed=5)
+    q, k = x["q"], x["k"]
+    nb = q.shape[1] // 64
+    exact = np.einsum("hid,hjd->hij", q.double().numpy().reshape(2, nb, 64, 128).mean(2),
+                      k.double().numpy().reshape(1, nb, 64, 128).mean(2).repeat(2, 0))
+    bound = bs_score_bound(q, k)
+    assert BS_TC_ERR_COEF < BS_ERR_COEF  # inside the index band's floor
+    err = np.abs(tc_pooled_scores_model(q, k) - exact)
+    assert np.all(err <= bound)
+    # dropping a part product the kernel forms (hi.mid) breaks the bound: the
+    # model is tight enough to see a missing term
+    err_drop = np.abs(tc_pooled_scores_model(q, k, ("hl", "mm", "lh", "mh", "hh")) - exact)
+    assert np.any(err_drop > bound)
