@@ -311,9 +311,6 @@ cudaError_t encode_attn_maps(AttnParams &P, const void *q, const void *k, const 
     return e;
 }
 
-// Work-item counters of the header, one per attention launch of a call.
-enum : int { SCHED_DENSE = 0, SCHED_VS = 1, SCHED_BLOCK = 2, SCHED_ASHAPE = 3, SCHED_TRISHAPE = 4 };
-
 int reset_counters(void *ws, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(static_cast<char *>(ws) + offsetof(WsHeader, tiles), 0,
                                     sizeof(WsHeader) - offsetof(WsHeader, tiles), st);
@@ -419,7 +416,6 @@ int do_vs_attention(const Common &c, const void *q, const void *k, const void *v
     P.vs_bits_v = b.bits_v;
     P.bit_stride = b.stride;
     P.vs_tiles = tiles ? 1 : 0;
-    P.sched_slot = SCHED_VS;
     e = run_attention(PAT_VS, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "vs attention launch");
 }
@@ -462,14 +458,13 @@ int do_block_attention(const Common &c, const void *q, const void *k, const void
     P.bs_plan = b.plan;
     P.bs_cnt = b.cnt;
     P.bs_stride = b.stride;
-    P.sched_slot = SCHED_BLOCK;
     e = run_attention(PAT_BLOCK, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "block attention launch");
 }
 
 int do_static_attention(int pattern, const Common &c, const void *q, const void *k, const void *v, float scale,
                         int n_sink, int window, int n_last, void *out, float *lse, void *ws, bool slot_is_id,
-                        int sched_slot, cudaStream_t st) {
+                        cudaStream_t st) {
     AttnParams P;
     memset(&P, 0, sizeof(P));
     fill_attn_common(P, c, scale, k, v, out, lse, ws, slot_is_id);
@@ -478,7 +473,6 @@ int do_static_attention(int pattern, const Common &c, const void *q, const void 
     P.n_sink = n_sink;
     P.window = window;
     P.n_last = n_last;
-    P.sched_slot = sched_slot;
     e = run_attention(pattern, P, st);
     return e == cudaSuccess ? MINF_OK : cuda_fail(e, "attention launch");
 }
@@ -705,7 +699,7 @@ int minf_ashape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf1
     if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
-    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, 0, out, lse, ws, false, SCHED_ASHAPE,
+    return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, 0, out, lse, ws, false,
                                (cudaStream_t)stream);
 }
 
@@ -725,7 +719,7 @@ int minf_trishape_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_b
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
     return do_static_attention(PAT_ASHAPE, c, q, k, v, scale, n_sink, window, n_last, out, lse, ws, false,
-                               SCHED_TRISHAPE, (cudaStream_t)stream);
+                               (cudaStream_t)stream);
 }
 
 int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
@@ -740,8 +734,7 @@ int minf_dense_attention(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16
     if ((rc = check_ws(ws, ws_bytes, MINF_STATUS_BYTES))) return rc;
     if ((rc = select_device(q))) return rc;
     if ((rc = reset_counters(ws, (cudaStream_t)stream))) return rc;
-    return do_static_attention(PAT_DENSE, c, q, k, v, scale, 0, 1, 0, out, lse, ws, false, SCHED_DENSE,
-                               (cudaStream_t)stream);
+    return do_static_attention(PAT_DENSE, c, q, k, v, scale, 0, 1, 0, out, lse, ws, false, (cudaStream_t)stream);
 }
 
 int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v, int hq, int hkv, int n, int d,
@@ -818,13 +811,12 @@ int minf_mixed_layer(const minf_bf16 *q, const minf_bf16 *k, const minf_bf16 *v,
     }
     if (!rc && sub[PAT_ASHAPE].n_heads)
         rc = do_static_attention(PAT_ASHAPE, sub[PAT_ASHAPE], q, k, v, scale, n_sink, window, 0, out, lse, ws, true,
-                                 SCHED_ASHAPE, st);
+                                 st);
     if (!rc && sub[MINF_PATTERN_TRISHAPE].n_heads)
         rc = do_static_attention(PAT_ASHAPE, sub[MINF_PATTERN_TRISHAPE], q, k, v, scale, n_sink, window, last_q, out,
-                                 lse, ws, true, SCHED_TRISHAPE, st);
+                                 lse, ws, true, st);
     if (!rc2 && sub[PAT_DENSE].n_heads)
-        rc2 = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, 0, out, lse, ws, true,
-                                  SCHED_DENSE, st2);
+        rc2 = do_static_attention(PAT_DENSE, sub[PAT_DENSE], q, k, v, scale, 0, 1, 0, out, lse, ws, true, st2);
     if (two) {
         // join even after a failed launch: nothing may stay queued behind the caller's back
         cudaError_t e = cudaEventRecord(ev_side, side);

@@ -25,8 +25,6 @@
 // straight from TMEM (TS MMA).  The running max only moves when a row's max
 // grows by more than 2^8.  A build-time share of the exponentials can run on
 // the FMA pipe (polynomial) instead of the MUFU unit.
-#include <algorithm>
-
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -43,13 +41,7 @@ constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kTileBytes;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
 constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
-constexpr uint32_t kSmemEx = kSmemBar + 256;                 // epilogue (max, sum) exchange, 256 float2
-constexpr uint32_t kSmemUsed = kSmemEx + 2048;
-// The dynamic shared memory is declared 1024-byte aligned; the kernel still rounds
-// its base up and checks that the rounding fits this slack.
-constexpr uint32_t kSmemSlack = 256;
-constexpr uint32_t kSmemBytes = kSmemUsed + kSmemSlack;
-static_assert(kSmemBytes <= 232448, "fits the per-CTA shared-memory limit");
+constexpr uint32_t kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
 // Register split after setmaxnreg: the launch gives 384 threads x 168 registers;
 // the load/MMA warpgroup drops to 56, the two softmax warpgroups rise to 224
 // (128 x 56 + 256 x 224 = 384 x 168).
@@ -72,12 +64,8 @@ constexpr int kEmuEvery = MINF_EMU_EVERY;
 
 enum : int {
     B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 4, B_V_FULL = 7, B_V_EMPTY = 10,
-    B_S_FULL = 13, B_P_FULL = 15, B_ALL_DONE = 17, B_Q_EMPTY = 18, B_O_FREE = 19,
-    B_ITEM_FULL = 20, B_ITEM_EMPTY = 22, B_FIN = 24, B_COUNT = 25
+    B_S_FULL = 13, B_P_FULL = 15, B_ALL_DONE = 17, B_COUNT = 18
 };
-// Warps that read each work item from the ring: the V producer, the MMA warp and
-// the eight softmax warps.
-constexpr int kItemReaders = 10;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, true);
@@ -341,48 +329,32 @@ __device__ __forceinline__ void exp2_poly_pair(float &a, float &b) {
     f32x2_unpack(p, a, b);
 }
 
-// Work item idx of the launch order: query tile t of head position hp.
-struct Item {
-    int t, hp;
-};
-__device__ __forceinline__ Item item_at(const AttnParams &P, int idx) {
-    int gi = 0;
-    while (gi + 1 < P.n_kvgroups && idx >= P.kv_start[gi + 1] * P.n_qtiles) ++gi;
-    const int gh = P.kv_start[gi + 1] - P.kv_start[gi];
-    const int local = idx - P.kv_start[gi] * P.n_qtiles;
-    return Item{P.n_qtiles - 1 - local / gh, P.kv_order[P.kv_start[gi] + local % gh]};
-}
-
-// Persistent: one CTA per SM takes work items in launch order from a counter in
-// the workspace header (the K producer draws them and hands them to the other
-// roles through a two-slot ring), so the items stay heaviest first and an SM
-// that finishes early takes the next one.  Rings, S/P buffers and their barrier
-// phases run on across items; one item's epilogue overlaps the next item's Q,
-// K and V loads and first S products.
 template <int PAT>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    if (smem - smem_raw > (ptrdiff_t)kSmemSlack) {
-        // the swizzled stages need 1024-byte alignment that the launch did not give:
-        // report it and do nothing (every thread takes this branch)
-        if (threadIdx.x == 0 && P.hdr) atomicExch(&P.hdr->status, MINF_ERR_CUDA);
-        return;
-    }
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sQ = sbase + kSmemQ, sK = sbase + kSmemK, sV = sbase + kSmemV;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + B_COUNT);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT + 1);
-    volatile int *item_slot = reinterpret_cast<volatile int *>(bars + B_COUNT + 2);  // two entries
     auto bar = [&](int i) { return smem_u32(bars + i); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = P.n_heads * P.n_qtiles;
+    // groups of heads one after the other; within a group the heaviest query tiles first,
+    // its heads side by side
+    int gi = 0;
+    while (gi + 1 < P.n_kvgroups && (int)blockIdx.x >= P.kv_start[gi + 1] * P.n_qtiles) ++gi;
+    const int gh = P.kv_start[gi + 1] - P.kv_start[gi];
+    const int local = (int)blockIdx.x - P.kv_start[gi] * P.n_qtiles;
+    const int t = P.n_qtiles - 1 - local / gh;
+    const int hp = P.kv_order[P.kv_start[gi] + local % gh];
+    const int h = P.head_ids[hp];
+    const int g = h / P.group;
+    const int w_item = hp * P.n_qtiles + t;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q_FULL), 1);
-        mbar_init(bar(B_Q_EMPTY), 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(B_K_FULL + s), 1);
             mbar_init(bar(B_K_EMPTY + s), 1);
@@ -392,12 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_S_FULL + b), 1);
             mbar_init(bar(B_P_FULL + b), 128);
-            mbar_init(bar(B_ITEM_FULL + b), 1);
-            mbar_init(bar(B_ITEM_EMPTY + b), kItemReaders);
         }
         mbar_init(bar(B_ALL_DONE), 1);
-        mbar_init(bar(B_O_FREE), 8);
-        mbar_init(bar(B_FIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -416,16 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const uint32_t tmem = *tmem_slot;
     const WaitCtl wc{abort_flag, P.hdr ? &P.hdr->status : nullptr, P.wait_limit_ns};
 
-    // a consumer warp's next item index (n_items or more: no more work; -1: gave up)
-    auto take_item = [&](int seq) -> int {
-        const int s = seq & 1;
-        const bool got = wait_bounded(bar(B_ITEM_FULL + s), (seq >> 1) & 1, wc, wait_site(13, B_ITEM_FULL + s, seq));
-        if (__any_sync(0xffffffffu, !got)) return -1;
-        const int idx = item_slot[s];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + s));
-        return idx;
-    };
+    TileGen<PAT> gen;
+    gen.init(P, hp, t);
+    const int T = gen.tiles();
+    const int *vlist = nullptr;
+    if constexpr (PAT == PAT_VS) vlist = P.vs_vert + (size_t)w_item * P.vs_vstride;
 
     if (warp < 4) {
         // ---------------------------------------------------------- load / MMA warpgroup
@@ -436,309 +399,206 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const __nv_bfloat16 *raw = is_k ? P.k : P.v;
             const uint32_t stage0 = is_k ? sK : sV;
             const int full0 = is_k ? B_K_FULL : B_V_FULL, empty0 = is_k ? B_K_EMPTY : B_V_EMPTY;
-            uint32_t jrun = 0, issued = 0;  // tiles of this CTA so far; tiles whose load was issued
-            int qn = 0;                     // items with tiles so far (Q loads)
-            bool ok = true;
-            for (int seq = 0; ok; ++seq) {
-                int idx;
-                if (is_k) {
-                    // draw the next item and hand it to the other roles
-                    const int s = seq & 1;
-                    ok = !__any_sync(0xffffffffu, !wait_bounded(bar(B_ITEM_EMPTY + s), ((seq >> 1) & 1) ^ 1, wc,
-                                                                wait_site(1, B_ITEM_EMPTY + s, seq)));
-                    if (!ok) break;
-                    idx = 0;
-                    if (lane == 0) {
-                        idx = (int)atomicAdd(&P.hdr->sched[P.sched_slot], 1u);
-                        item_slot[s] = idx;
-                        mbar_arrive(bar(B_ITEM_FULL + s));
-                    }
-                    idx = __shfl_sync(0xffffffffu, idx, 0);
-                } else {
-                    idx = take_item(seq);
-                    if (idx < 0) break;
-                }
-                if (idx >= n_items) break;
-                const Item it = item_at(P, idx);
-                const int h = P.head_ids[it.hp], g = h / P.group;
-                TileGen<PAT> gen;
-                gen.init(P, it.hp, it.t);
-                const int T = gen.tiles();
-                const int *vlist = nullptr;
-                if constexpr (PAT == PAT_VS) vlist = P.vs_vert + (size_t)(it.hp * P.n_qtiles + it.t) * P.vs_vstride;
-                if (is_k && T > 0) {
-                    // the Q stage is free once every S product of the previous item with tiles has completed
-                    ok = !__any_sync(0xffffffffu, !wait_bounded(bar(B_Q_EMPTY), (qn & 1) ^ 1, wc,
-                                                                wait_site(1, B_Q_EMPTY, qn)));
-                    if (!ok) break;
-                    const int r0 = it.t * kTileM;
-                    tma_load_stage_warp(sQ, &P.tmap_q, bar(B_Q_FULL), 4 * 8192, r0, r0 + 64, h, 3u);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_Q_FULL));
-                }
-                if (T > 0) ++qn;
-                for (int j = 0; j < T; ++j, ++jrun) {
-                    const int s = jrun % kStages;
-                    const uint32_t ph = (jrun / kStages) & 1;
-                    HalfDesc hd[2];
-                    hd[0] = gen.next(P);
-                    hd[1] = gen.next(P);
-                    // one decision per warp: every lane takes the same path through load_tile
-                    const bool got = wait_bounded(bar(empty0 + s), ph ^ 1, wc, wait_site(is_k ? 1 : 2, empty0 + s, j));
-                    if (__any_sync(0xffffffffu, !got)) {
-                        ok = false;
-                        break;
-                    }
-                    load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
-                    issued = jrun + 1;
-                }
+            if (is_k && T > 0) {
+                const int r0 = t * kTileM;
+                tma_load_stage_warp(sQ, &P.tmap_q, bar(B_Q_FULL), 4 * 8192, r0, r0 + 64, h, 3u);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_Q_FULL));
+            }
+            int issued = 0;
+            for (int j = 0; j < T; ++j) {
+                const int s = j % kStages;
+                const uint32_t ph = (j / kStages) & 1;
+                HalfDesc hd[2];
+                hd[0] = gen.next(P);
+                hd[1] = gen.next(P);
+                // one decision per warp: every lane takes the same path through load_tile
+                const bool got = wait_bounded(bar(empty0 + s), ph ^ 1, wc, wait_site(is_k ? 1 : 2, empty0 + s, j));
+                if (__any_sync(0xffffffffu, !got)) break;
+                load_tile<PAT>(stage0 + s * kTileBytes, bar(full0 + s), hd, map, raw, g, P.n, vlist, lane);
+                issued = j + 1;
             }
             if (*abort_flag && lane == 0) {
                 // drain: let the loads already issued land before the CTA exits
                 volatile int no_abort = 0;
                 const WaitCtl drain{&no_abort, nullptr, 50000000ull};
-                for (uint32_t j = issued > (uint32_t)kStages ? issued - kStages : 0u; j < issued; ++j)
+                for (int j = max(0, issued - kStages); j < issued; ++j)
                     wait_bounded(bar(full0 + j % kStages), (j / kStages) & 1, drain);
-                if (is_k && qn > 0) wait_bounded(bar(B_Q_FULL), (qn - 1) & 1, drain);
             }
-        } else if (warp == 1) {
-            // tcgen05 issue: S(J) = Q K(J)^T into S[J % 2]; O[J % 2] += P(J) V(J) with P(J)
-            // read from the first 64 columns of S[J % 2] (J counts the CTA's tiles); within an
-            // item S(j + 2) is issued after P(j) V(j) and the tensor pipe runs them in order,
-            // so P(j) is consumed before it is overwritten.  The whole warp runs this loop
-            // (waits, counters and descriptors stay warp-uniform); elect.sync picks the lane
-            // that issues.  Step-0 descriptors of Q, K stage 0 and V stage 0; a stage adds its
-            // offset / 16.
+        } else if (warp == 1 && T > 0) {
+            // tcgen05 issue: S(j) = Q K(j)^T into S[j % 2]; O[j % 2] += P(j) V(j) with P(j)
+            // read from the first 64 columns of S[j % 2]; S(j + 2) is issued after P(j) V(j)
+            // and the tensor pipe runs them in order, so P(j) is consumed before it is overwritten.
+            // The whole warp runs this loop (waits, counters and descriptors stay warp-uniform,
+            // every decision is taken by the warp as one); elect.sync picks the lane that issues.
+            // step-0 descriptors of Q, K stage 0 and V stage 0; a stage adds its offset / 16
             const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
             const uint64_t dv0 = sdesc_sw128(sV, 16384, 1024);
-            uint32_t jrun = 0;
-            int qn = 0;
-            unsigned long long my_tiles = 0;
-            bool ok = true;
-            for (int seq = 0; ok; ++seq) {
-                const int idx = take_item(seq);
-                if (idx < 0 || idx >= n_items) break;
-                const Item it = item_at(P, idx);
-                TileGen<PAT> gen;
-                gen.init(P, it.hp, it.t);
-                const int T = gen.tiles();
-                // O may be overwritten once the previous item's epilogue has read it
-                auto wait_o_free = [&]() -> bool {
-                    if (seq == 0) return true;
-                    return __all_sync(0xffffffffu, wait_bounded(bar(B_O_FREE), (seq - 1) & 1, wc,
-                                                                wait_site(3, B_O_FREE, seq)));
-                };
-                auto issue_s = [&](int j) -> bool {
-                    const uint32_t J = jrun + j;
-                    const int s = J % kStages;
-                    const bool got = wait_bounded(bar(B_K_FULL + s), (J / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j));
-                    if (!__all_sync(0xffffffffu, got)) return false;
-                    tc_fence_after();
-                    umma_ss_tile_warp(tmem + (J & 1) * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
-                    umma_commit_warp(bar(B_K_EMPTY + s));
-                    umma_commit_warp(bar(B_S_FULL + (J & 1)));
-                    if (j == T - 1) umma_commit_warp(bar(B_Q_EMPTY));  // the item's last use of Q
-                    return true;
-                };
-                if (T > 0) {
-                    ok = __all_sync(0xffffffffu, wait_bounded(bar(B_Q_FULL), qn & 1, wc, wait_site(3, B_Q_FULL, qn)));
-                    ++qn;
-                    if (ok) {
-                        tc_fence_after();
-                        ok = issue_s(0);
-                        if (ok && T > 1) ok = issue_s(1);
-                    }
-                    for (int j = 0; ok && j < T; ++j) {
-                        const uint32_t J = jrun + j;
-                        const int b = J & 1, s = J % kStages;
-                        bool got = wait_bounded(bar(B_P_FULL + b), (J >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j));
-                        if (!__all_sync(0xffffffffu, got)) {
-                            ok = false;
-                            break;
-                        }
-                        got = wait_bounded(bar(B_V_FULL + s), (J / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j));
-                        if (!__all_sync(0xffffffffu, got) || (j == 0 && !wait_o_free())) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        umma_ts_tile_warp(tmem + 256 + b * 128, tmem + b * 128, dv0 + (uint64_t)((s * kTileBytes) >> 4),
-                                          kIdescPV, j >= 2 ? 1u : 0u);
-                        umma_commit_warp(bar(B_V_EMPTY + s));
-                        if (j + 2 < T && !issue_s(j + 2)) {
-                            ok = false;
-                            break;
-                        }
-                    }
-                    jrun += T;
-                } else {
-                    // nothing to compute: hand over as soon as the previous epilogue is done
-                    ok = wait_o_free();
-                }
-                if (!ok) break;
-                umma_commit_warp(bar(B_ALL_DONE));  // the item's products are complete: its epilogue may run
-                my_tiles += T;
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % kStages;
+                const bool got = wait_bounded(bar(B_K_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_K_FULL + s, j));
+                if (!__all_sync(0xffffffffu, got)) return false;
+                tc_fence_after();
+                umma_ss_tile_warp(tmem + (j & 1) * 128, dq, dk0 + (uint64_t)((s * kTileBytes) >> 4), kIdescQK, 0u);
+                umma_commit_warp(bar(B_K_EMPTY + s));
+                umma_commit_warp(bar(B_S_FULL + (j & 1)));
+                return true;
+            };
+            bool ok = __all_sync(0xffffffffu, wait_bounded(bar(B_Q_FULL), 0, wc, wait_site(3, B_Q_FULL, 0)));
+            if (ok) {
+                tc_fence_after();
+                ok = issue_s(0);
+                if (ok && T > 1) ok = issue_s(1);
             }
-            if (P.hdr && lane == 0 && my_tiles) {
-                atomicAdd(&P.hdr->tiles, my_tiles);
-                atomicAdd(&P.hdr->pat_tiles[PAT], my_tiles);
+            for (int j = 0; ok && j < T; ++j) {
+                const int b = j & 1, s = j % kStages;
+                bool got = wait_bounded(bar(B_P_FULL + b), (j >> 1) & 1, wc, wait_site(3, B_P_FULL + b, j));
+                if (!__all_sync(0xffffffffu, got)) break;
+                got = wait_bounded(bar(B_V_FULL + s), (j / kStages) & 1, wc, wait_site(3, B_V_FULL + s, j));
+                if (!__all_sync(0xffffffffu, got)) break;
+                tc_fence_after();
+                umma_ts_tile_warp(tmem + 256 + b * 128, tmem + b * 128, dv0 + (uint64_t)((s * kTileBytes) >> 4),
+                                  kIdescPV, j >= 2 ? 1u : 0u);
+                umma_commit_warp(bar(B_V_EMPTY + s));
+                if (j + 2 < T && !issue_s(j + 2)) break;
             }
-            // every product issued has completed before TMEM is freed
-            umma_commit_warp(bar(B_FIN));
-            volatile int no_abort = 0;
-            const WaitCtl drain{&no_abort, nullptr, 50000000ull};
-            wait_bounded(bar(B_FIN), 0, drain);
+            umma_commit_warp(bar(B_ALL_DONE));  // always close: the epilogue (or the abort path) waits on it
+            if (P.hdr && lane == 0) {
+                atomicAdd(&P.hdr->tiles, (unsigned long long)T);
+                atomicAdd(&P.hdr->pat_tiles[PAT], (unsigned long long)T);
+            }
         }
     } else {
         // ---------------------------------------------------------- softmax warpgroups
         setmaxnreg_inc<kRegsSoftmax>();
-        const int wg = (warp - 4) >> 2;          // S/O buffer of this warpgroup: tiles J with J % 2 == wg
-        const int r = (threadIdx.x - 128) & 127; // query row within the tile = TMEM lane
+        const int wg = (warp - 4) >> 2;          // 0: even tiles, 1: odd tiles
+        const int r = (threadIdx.x - 128) & 127; // query row = TMEM lane
+        const int q = t * kTileM + r;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + wg * 128;
         const uint32_t tO = tmem + lane_off + 256 + wg * 128;
         const float sl2 = P.scale_log2;
-        float2 *ex = reinterpret_cast<float2 *>(smem + kSmemEx);
+        const uint32_t *bits_s = nullptr, *bits_v = nullptr;
+        if constexpr (PAT == PAT_VS) {
+            bits_s = P.vs_bits_s + (size_t)hp * P.bit_stride;
+            bits_v = P.vs_bits_v + (size_t)hp * P.bit_stride;
+        }
+        float m_run = -INFINITY, l_run = 0.f;
         unsigned long long pairs = 0;
-        uint32_t jrun = 0;
-        for (int seq = 0;; ++seq) {
-            const int idx = take_item(seq);
-            // every softmax warp leaves the loop at the same item: the named barriers
-            // below must see all eight warps or none
-            if (named_bar_or(2, 256, idx < 0 || idx >= n_items)) break;
-            const Item it = item_at(P, idx);
-            const int t = it.t, hp = it.hp;
-            const int q = t * kTileM + r;
-            TileGen<PAT> gen;
-            gen.init(P, hp, t);
-            const int T = gen.tiles();
-            const int *vlist = nullptr;
-            const uint32_t *bits_s = nullptr, *bits_v = nullptr;
-            if constexpr (PAT == PAT_VS) {
-                vlist = P.vs_vert + (size_t)(it.hp * P.n_qtiles + it.t) * P.vs_vstride;
-                bits_s = P.vs_bits_s + (size_t)hp * P.bit_stride;
-                bits_v = P.vs_bits_v + (size_t)hp * P.bit_stride;
-            }
-            const int jf = (int)((wg - jrun) & 1u);  // this warpgroup's first tile of the item
-            float m_run = -INFINITY, l_run = 0.f;
-            bool ok = true;
-            if (jf == 1) gen.skip2(P);  // tile 0 belongs to the other warpgroup
-            // element masks of this warpgroup's next tile: described, their bitmap words
-            // loaded and combined while the warpgroup waits for that tile's S, so that
-            // only the two 64-bit masks stay live through the softmax
-            uint64_t mk0 = 0, mk1 = 0;
-            bool full = false;
-            auto prepare = [&]() {
-                const HalfDesc d0 = gen.next(P), d1 = gen.next(P);
-                MaskWords w0, w1;
-                mask_fetch<PAT>(P, d0, q, bits_s, bits_v, w0);
-                mask_fetch<PAT>(P, d1, q, bits_s, bits_v, w1);
-                mk0 = half_mask<PAT>(P, d0, q, r, vlist, w0);
-                mk1 = half_mask<PAT>(P, d1, q, r, vlist, w1);
-                full = (d0.flags & d1.flags & HF_FULL) != 0;  // uniform over the CTA
-            };
-            prepare();
-            for (int j = jf; j < T; j += 2) {
-                const uint32_t J = jrun + j;
-                if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
-                const bool got = wait_bounded(bar(B_S_FULL + wg), (J >> 1) & 1, wc, wait_site(4 + wg, B_S_FULL + wg, j));
-                if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // tcgen05.ld below is warp-wide
-                tc_fence_after();
-                uint32_t sr[4][32];
+        bool ok = true;
+        if (wg == 1) gen.skip2(P);  // tile 0 belongs to the other warpgroup
+        // element masks of this warpgroup's next tile: described, their bitmap words
+        // loaded and combined while the warpgroup waits for that tile's S, so that
+        // only the two 64-bit masks stay live through the softmax
+        uint64_t mk0 = 0, mk1 = 0;
+        bool full = false;
+        auto prepare = [&]() {
+            const HalfDesc d0 = gen.next(P), d1 = gen.next(P);
+            MaskWords w0, w1;
+            mask_fetch<PAT>(P, d0, q, bits_s, bits_v, w0);
+            mask_fetch<PAT>(P, d1, q, bits_s, bits_v, w1);
+            mk0 = half_mask<PAT>(P, d0, q, r, vlist, w0);
+            mk1 = half_mask<PAT>(P, d1, q, r, vlist, w1);
+            full = (d0.flags & d1.flags & HF_FULL) != 0;  // uniform over the CTA
+        };
+        prepare();
+        for (int j = wg; j < T; j += 2) {
+            if (q < P.n) pairs += __popcll(mk0) + __popcll(mk1);
+            const bool got = wait_bounded(bar(B_S_FULL + wg), (j >> 1) & 1, wc, wait_site(4 + wg, B_S_FULL + wg, j));
+            if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // tcgen05.ld below is warp-wide
+            tc_fence_after();
+            uint32_t sr[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-                if (!full) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t mw = (uint32_t)((c < 2 ? mk0 : mk1) >> ((c & 1) * 32));
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!((mw >> e) & 1u)) sr[c][e] = 0xff800000u;  // -inf
-                    }
-                }
-                // row max over the 128 columns: four independent three-input max chains
-                float mc[4];
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+            if (!full) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+                    const uint32_t mw = (uint32_t)((c < 2 ? mk0 : mk1) >> ((c & 1) * 32));
 #pragma unroll
-                    for (int e = 2; e < 32; e += 2)
-                        mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                    for (int e = 0; e < 32; ++e)
+                        if (!((mw >> e) & 1u)) sr[c][e] = 0xff800000u;  // -inf
                 }
-                float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
-                mx *= sl2;
-                const float m_new = fmaxf(m_run, mx);
-                const bool want = m_new > m_run + 8.0f;  // includes m_run = -inf with a finite m_new
-                const float alpha = want ? ex2_approx(m_run - m_new) : 1.f;  // 0 when m_run = -inf
-                // O[wg] holds this warpgroup's tiles < j of the item, all complete (S(j) was
-                // issued after their P.V): rescale it in TMEM with the whole warp (lanes that
-                // keep their max use alpha = 1)
-                if (j >= 2 && __any_sync(0xffffffffu, want && m_run != -INFINITY)) {
+            }
+            // row max over the 128 columns: four independent three-input max chains
+            float mc[4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-                        tmem_ld_wait(o);
+            for (int c = 0; c < 4; ++c) {
+                mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tO + c * 32, o);
-                    }
-                }
-                if (want) {
-                    l_run *= alpha;
-                    m_run = m_new;
-                }
-                const float m_use = m_run == -INFINITY ? 0.f : m_run;
-                const uint64_t sl2x2 = f32x2_splat(sl2), negm = f32x2_splat(-m_use);
-                uint64_t acc0 = 0, acc1 = 0;  // two running (sum, sum) pairs
-                uint32_t pp[2][32];
+                for (int e = 2; e < 32; e += 2)
+                    mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+            }
+            float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+            mx *= sl2;
+            const float m_new = fmaxf(m_run, mx);
+            const bool want = m_new > m_run + 8.0f;  // includes m_run = -inf with a finite m_new
+            const float alpha = want ? ex2_approx(m_run - m_new) : 1.f;  // 0 when m_run = -inf
+            // O[wg] holds this warpgroup's tiles < j, all complete (S(j) was issued after their P.V):
+            // rescale it in TMEM with the whole warp (lanes that keep their max use alpha = 1)
+            if (j >= 2 && __any_sync(0xffffffffu, want && m_run != -INFINITY)) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait(o);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
-                                                     sl2x2, negm);
-                        float p0, p1;
-                        f32x2_unpack(x, p0, p1);
-                        if (kEmuEvery > 0 && (e % kEmuEvery) == kEmuEvery - 1) {
-                            exp2_poly_pair(p0, p1);
-                        } else {
-                            p0 = ex2_approx(p0);
-                            p1 = ex2_approx(p1);
-                        }
-                        if (e & 1) acc1 = f32x2_add(acc1, f32x2_pack(p0, p1));
-                        else acc0 = f32x2_add(acc0, f32x2_pack(p0, p1));
-                        pp[c >> 1][(c & 1) * 16 + e] = pack_bf16x2(p0, p1);
-                    }
-                    if (c == 1) tmem_st32(tS, pp[0]);  // P(j) columns 0-31 of S[wg], stored while 32-63 are computed
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + c * 32, o);
                 }
-                float a0, a1, b0, b1;
-                f32x2_unpack(acc0, a0, a1);
-                f32x2_unpack(acc1, b0, b1);
-                l_run += (a0 + a1) + (b0 + b1);
-                tmem_st32(tS + 32, pp[1]);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(bar(B_P_FULL + wg));
-                gen.skip2(P);  // the other warpgroup's tile j + 1
-                prepare();     // tile j + 2
             }
-            // ------------------------------------------------------------ epilogue
-            ok = __all_sync(0xffffffffu, ok);
-            if (ok) ok = wait_bounded(bar(B_ALL_DONE), seq & 1, wc, wait_site(4 + wg, B_ALL_DONE, seq));
-            // one decision for all eight warps (the TMEM loads below are warp-wide, the
-            // barriers below CTA-wide over the softmax warps)
-            if (named_bar_or(1, 256, !ok)) break;
-            // exchange (max, sum) of the two halves of the key stream through shared memory
-            ex[wg * 128 + r] = make_float2(m_run, l_run);
-            named_bar_sync(1, 256);
+            if (want) {
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            const float m_use = m_run == -INFINITY ? 0.f : m_run;
+            const uint64_t sl2x2 = f32x2_splat(sl2), negm = f32x2_splat(-m_use);
+            uint64_t acc0 = 0, acc1 = 0;  // two running (sum, sum) pairs
+            uint32_t pp[2][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                                                 sl2x2, negm);
+                    float p0, p1;
+                    f32x2_unpack(x, p0, p1);
+                    if (kEmuEvery > 0 && (e % kEmuEvery) == kEmuEvery - 1) {
+                        exp2_poly_pair(p0, p1);
+                    } else {
+                        p0 = ex2_approx(p0);
+                        p1 = ex2_approx(p1);
+                    }
+                    if (e & 1) acc1 = f32x2_add(acc1, f32x2_pack(p0, p1));
+                    else acc0 = f32x2_add(acc0, f32x2_pack(p0, p1));
+                    pp[c >> 1][(c & 1) * 16 + e] = pack_bf16x2(p0, p1);
+                }
+                if (c == 1) tmem_st32(tS, pp[0]);  // P(j) columns 0-31 of S[wg], stored while 32-63 are computed
+            }
+            float a0, a1, b0, b1;
+            f32x2_unpack(acc0, a0, a1);
+            f32x2_unpack(acc1, b0, b1);
+            l_run += (a0 + a1) + (b0 + b1);
+            tmem_st32(tS + 32, pp[1]);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(B_P_FULL + wg));
+            gen.skip2(P);  // the other warpgroup's tile j + 1
+            prepare();     // tile j + 2
+        }
+        // ------------------------------------------------------------ epilogue
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && T > 0) ok = wait_bounded(bar(B_ALL_DONE), 0, wc, wait_site(4 + wg, B_ALL_DONE, T));
+        ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-wide
+        // exchange (max, sum) of the two halves of the key stream through shared memory
+        // (the K stages are idle once every MMA has completed)
+        float2 *ex = reinterpret_cast<float2 *>(smem + kSmemK);
+        ex[wg * 128 + r] = make_float2(m_run, l_run);
+        named_bar_sync(1, 256);
+        if (ok) {
             tc_fence_after();
             const float2 s0 = ex[r], s1 = ex[128 + r];
-            named_bar_sync(1, 256);  // both read before either warpgroup writes the next item's
-            // buffer b holds data of this item iff warpgroup b had a tile in it
-            const bool has0 = T > (int)(jrun & 1u), has1 = T > (int)((jrun + 1u) & 1u);
             // a third partial state: the row's sparse-slash pairs, from the CUDA-core pass
             float2 s2 = make_float2(-INFINITY, 0.f);
             if constexpr (PAT == PAT_VS) {
@@ -746,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             const bool has2 = s2.y > 0.f;
             const float m = fmaxf(fmaxf(s0.x, s1.x), has2 ? s2.x : -INFINITY);
-            const float a0 = (!has0 || s0.x == -INFINITY) ? 0.f : ex2_approx(s0.x - m);
-            const float a1 = (!has1 || s1.x == -INFINITY) ? 0.f : ex2_approx(s1.x - m);
+            const float a0 = s0.x == -INFINITY ? 0.f : ex2_approx(s0.x - m);
+            const float a1 = (T < 2 || s1.x == -INFINITY) ? 0.f : ex2_approx(s1.x - m);
             const float a2 = has2 ? ex2_approx(s2.x - m) : 0.f;
             const float l = s0.y * a0 + s1.y * a1 + s2.y * a2;
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -760,25 +620,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t o0[32], o1[32];
-                if (has0) {  // uniform over the CTA
+                if (T > 0) {  // uniform over the CTA
                     tmem_ld32(tO0 + c * 32, o0);
                     tmem_ld_wait(o0);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o0[e] = 0u;
                 }
-                if (has1) {
+                if (T > 1) {
                     tmem_ld32(tO1 + c * 32, o1);
                     tmem_ld_wait(o1);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o1[e] = 0u;
-                }
-                if (c == 1) {
-                    // O is in registers: the next item's P.V products may overwrite it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_O_FREE));
                 }
                 if (q < P.n) {
 #pragma unroll
@@ -803,8 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
-            if (wg == 0 && q < P.n && P.lse) P.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-            jrun += T;
+            if (wg == 0 && q < P.n && P.lse)
+                P.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
         if (P.hdr) {
 #pragma unroll
@@ -1066,15 +920,8 @@ cudaError_t launch_attn(const AttnParams &P, cudaStream_t st) {
     e = cudaFuncGetAttributes(&fa, attn_kernel<PAT>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-    // the work-item counter lives in the workspace header (zeroed at the call's start)
-    if (!P.hdr || P.sched_slot < 0 || P.sched_slot >= 8) return cudaErrorInvalidValue;
-    const int items = P.n_heads * P.n_qtiles;
-    if (items == 0) return cudaSuccess;
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    const int grid = std::min(items, std::max(sms, 1));  // one CTA per SM
+    const int grid = P.n_heads * P.n_qtiles;
+    if (grid == 0) return cudaSuccess;
     static const char *const names[] = {"attn_kernel<DENSE>", "attn_kernel<VS>", "attn_kernel<BLOCK>",
                                         "attn_kernel<ASHAPE>"};
     ProfScope prof(names[PAT], st);
@@ -1105,9 +952,6 @@ cudaError_t run_exp2_selftest(const float *x, float *y_poly, float *y_hw, int n,
 }
 
 cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st) {
-    // P.sched_slot: the caller's choice of work-item counter; launches of one call
-    // that may run at the same time or one after the other without a reset in
-    // between each take their own
     switch (pattern) {
     case PAT_DENSE: return launch_attn<PAT_DENSE>(P, st);
     case PAT_ASHAPE: return launch_attn<PAT_ASHAPE>(P, st);

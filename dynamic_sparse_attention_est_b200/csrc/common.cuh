@@ -27,7 +27,6 @@ struct WsHeader {
     unsigned long long pairs;
     unsigned long long pat_tiles[4];  // tiles by attention kernel pattern (PAT_*)
     unsigned long long diag_pairs;    // pairs of the CUDA-core sparse-slash pass (included in pairs)
-    unsigned sched[8];                // next work item of each persistent attention launch of a call
 };
 static_assert(sizeof(WsHeader) <= MINF_STATUS_BYTES, "header fits the status block");
 
@@ -91,7 +90,6 @@ struct AttnParams {
     // side.  Grouped by kv-head, the CTAs in flight share that kv-head's K and V
     // in L2; a single group is the plain heaviest-first order.
     int n_kvgroups;
-    int sched_slot;                     // this launch's work-item counter in hdr->sched
     int kv_order[MINF_MAX_HEADS];       // head positions sorted by kv-head
     int kv_start[MINF_MAX_HEADS + 1];   // kv_order index where each group starts
 };
