@@ -479,8 +479,8 @@ int do_static_attention(int pattern, const Common &c, const void *q, const void 
 
 }  // namespace
 
-// TMA descriptor of a bf16 [heads][n][128] tensor, box {64, 64, 1}, 128-byte swizzle.
-cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n) {
+// The driver's tensor-map encoder, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult qres;
@@ -489,7 +489,12 @@ cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n) {
             qres == cudaDriverEntryPointSuccess)
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     });
-    if (!g_encode) return cudaErrorNotSupported;
+    return g_encode;
+}
+
+// TMA descriptor of a bf16 [heads][n][128] tensor, box {64, 64, 1}, 128-byte swizzle.
+cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n) {
+    if (!tmap_encoder()) return cudaErrorNotSupported;
     const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
     const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)n * kD * 2};
     const cuuint32_t box[3] = {64, 64, 1};
@@ -497,6 +502,20 @@ cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n) {
     const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// TMA descriptor of an fp32 [z][y][x] tensor (row stride x floats, a multiple of
+// 4), box {32, 32, 1}, 128-byte swizzle: the score tiles' store path.
+cudaError_t make_tmap_f32_3d(CUtensorMap *map, const void *base, int x, int y, int z) {
+    if (!tmap_encoder()) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)x, (cuuint64_t)y, (cuuint64_t)z};
+    const cuuint64_t strides[2] = {(cuuint64_t)x * 4, (cuuint64_t)x * y * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 

@@ -44,6 +44,7 @@ struct VsPlanBufs {
 
 // 3D TMA map over a bf16 [heads][n][128] tensor: box {64, 64, 1}, 128B swizzle.
 cudaError_t make_tmap_3d(CUtensorMap *map, const void *base, int heads, int n);
+cudaError_t make_tmap_f32_3d(CUtensorMap *map, const void *base, int x, int y, int z);
 
 cudaError_t run_attention(int pattern, const AttnParams &P, cudaStream_t st);
 cudaError_t run_bs_plan(const int *blk_idx, const int *blk_cnt, int topk, int n_heads, int n_qtiles, int nb,

@@ -155,6 +155,24 @@ __device__ __forceinline__ void tma_load_stage_warp(uint32_t dst, const void *tm
         "r"(dst + 16384), "r"(dst + 8192), "r"(dst + 16384 + 8192)
         : "memory");
 }
+// TMA store of one box from shared memory into a 3-D tensor (bulk-group completion:
+// bulk_commit closes the group, bulk_wait_read<N> waits until at most N groups of
+// this thread still read shared memory, bulk_wait<N> until at most N are
+// outstanding at all).  Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }

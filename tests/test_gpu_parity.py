@@ -85,6 +85,28 @@ def test_block_estimate_band(orc, n, hq, hkv, topk):
             assert np.all(gi[hp, i, gc[hp, i]:] == -1)
 
 
+@pytest.mark.parametrize("n_proto", [1, 3, 40])
+def test_block_estimate_exact_ties_go_to_lower_index(orc, n_proto):
+    """Key blocks copied from a few prototypes give pooled scores with exact ties
+    (bit-identical on both sides: identical operands, identical arithmetic), and
+    query blocks of zeros give rows of zeros.  The selection must then match the
+    oracle exactly, ties to the lower block index: with one prototype every row
+    is one tie (the whole row in one bin); with 3, each score value is shared by
+    about a third of the row (more than 32 candidates in the threshold bin: the
+    radix path); with 40, about 1/40 (the ranked path)."""
+    n, hq, hkv, topk = 64 * 300, 2, 1, 40
+    rng = np.random.default_rng(n_proto)
+    proto = rng.standard_normal((n_proto, 64, 128)).astype(np.float32)
+    pick = rng.integers(0, n_proto, n // 64)
+    k = torch.from_numpy(proto[pick].reshape(1, n, 128)).to(torch.bfloat16)
+    q = torch.from_numpy(rng.standard_normal((hq, n, 128)).astype(np.float32)).to(torch.bfloat16)
+    q[1, :64 * 20] = 0  # the first 20 query blocks of head 1: all-zero score rows
+    bi, bc = orc.block_estimate(q, k, 64, topk)
+    gi, gc = minf.minf_block_estimate(*cuda(q, k), topk=topk)
+    assert np.array_equal(gc.cpu().numpy(), bc)
+    assert np.array_equal(gi.cpu().numpy(), bi)
+
+
 @pytest.mark.parametrize("n,hq,hkv,ids", [(64 * 300, 4, 2, [3, 0, 2]),   # three row tiles, the last ragged
                                            (64 * 263, 2, 1, None),        # nb % 4 != 0: scalar stores
                                            (64 * 5, 2, 2, None)])         # one tile, fewer rows than a TMA box
