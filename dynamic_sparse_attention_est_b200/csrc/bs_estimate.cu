@@ -311,11 +311,12 @@ __global__ void __launch_bounds__(kScThreads, 1) pooled_scores_tc_kernel(const _
 //     their order-preserving keys (eight bits per pass, starting below the bits
 //     they all share, stopping once the digit holding the k-th is taken whole).
 // Rows up to kRowSmem scores are copied once into the warp's shared-memory row by
-// cp.async (the whole row in flight); one sweep then compacts the indices of bin
-// b* and above, in place, into a list in that row (candidates flagged), and the
-// output is taken from the list.  Longer rows, and bins of more than 32
-// candidates, are swept again for the output (re-read from L1/L2 when not
-// staged).  -0 is read as +0, so that equal scores have equal keys.
+// cp.async (the whole row in flight); longer rows are re-read (L1/L2) by every
+// sweep.  After the histogram one sweep compacts the indices of bin b* and above
+// into a list (candidates flagged) -- in place of a staged row, else in the
+// histogram's words -- and the output is taken from the list.  Bins of more than
+// 32 candidates (and, for long rows, budgets above 224) sweep the row again for
+// the output.  -0 is read as +0, so that equal scores have equal keys.
 constexpr int kTopkWarps = 8;
 constexpr int kRowSmem = 2048;
 
@@ -431,17 +432,19 @@ __device__ __forceinline__ void select_row(const float *src, float *row, int i, 
     __syncwarp();  // the histogram is read before it is reused below
     const bool all_of_bin = rem == in_bin;
     const bool ranked = !all_of_bin && in_bin <= 32;
-    if (STAGED && (all_of_bin || ranked)) {
-        // ---- one sweep: the indices of bin b* and above, compacted in place into the
-        // row (as float bits; bit 31 flags a candidate of b*), candidates also to `cand`
-        float *list = row;
+    // the list holds take - rem + in_bin <= take + 31 indices: staged rows keep it in
+    // place of the row, the others in the (no longer needed) histogram's 256 words
+    if ((all_of_bin || ranked) && (STAGED || take + 32 <= 256)) {
+        // ---- one sweep: the indices of bin b* and above, compacted into the list (as
+        // float bits; bit 31 flags a candidate of b*), candidates also to `cand`
+        float *list = STAGED ? row : reinterpret_cast<float *>(hist);
         int base = 0, cbase = 0;
-        row_sweep<true>(xs, i, lane, [&](int j, float x) {
+        row_sweep<STAGED>(xs, i, lane, [&](int j, float x) {
             const int b = j < i ? bin_of(x) : -1;
             const bool ge = b >= bstar, isc = b == bstar && !all_of_bin;
             const unsigned gm = __ballot_sync(0xffffffffu, ge), cm = __ballot_sync(0xffffffffu, isc);
-            // every lane has read its score before any lane writes (the ballots above
-            // depend on all the reads); positions written are <= this chunk's own
+            // staged: every lane has read its score before any lane writes (the ballots
+            // above depend on all the reads), and positions written are <= this chunk's own
             if (ge) list[base + __popc(gm & lt)] = __int_as_float(j | (isc ? (int)0x80000000 : 0));
             if (isc) cand[cbase + __popc(cm & lt)] = make_float2(x, __int_as_float(j));
             base += __popc(gm);
