@@ -9,7 +9,7 @@
 // another -- a 128-row query tile meets each offset in only one key per row, and
 // a 128x128 tile wastes 127 of every 128 products and exponentials.  This kernel
 // takes those groups instead: for each query tile it stages the groups' key
-// ranges in 64-key chunks (K and V, by TMA, as the tile kernel does), and each
+// ranges in 128-key chunks (K and V, by TMA, as the tile kernel does), and each
 // query row computes only its in-mask pairs, one dot product, one exponential
 // and one V update per offset (fp32 sums of products of bf16 operands).
 //
@@ -19,7 +19,7 @@
 // O -- which the tile kernel merges into its own in its epilogue.
 //
 // Roles (384 threads, one persistent CTA per SM striding over the work items):
-//   warp 0      TMA producer: one 64-key chunk of K and V per stage, 6 stages
+//   warp 0      TMA producer: one 128-key chunk of K and V per stage, 3 stages
 //   warps 1..3  idle (they give their registers to the consumers and exit)
 //   warps 4..11 consumers: two threads per query row (lane l of warp 4 + w holds
 //               row 16 w + (l & 15) and head dims [64 (l >> 4), 64 (l >> 4) + 64))
@@ -45,8 +45,9 @@ constexpr int kDiagRegsLaunch = 168;
 constexpr int kDiagRegsProducer = 40;
 constexpr int kDiagRegsConsumer = 232;
 static_assert(128 * kDiagRegsProducer + 256 * kDiagRegsConsumer <= kDiagThreads * kDiagRegsLaunch, "register split");
-constexpr int kDiagStages = 6;
-constexpr uint32_t kChunkBytes = 32768;  // 64 keys x 128 dims x 2 B, K then V
+constexpr int kDiagStages = 3;
+constexpr int kChunkKeys = 128;
+constexpr uint32_t kChunkBytes = 65536;  // 128 keys x 128 dims x 2 B, K then V
 constexpr uint32_t kDiagSmem = kDiagStages * kChunkBytes + 256 + 1024;  // + barriers + alignment slack
 
 // (acc0, acc1) += (lo(a) lo(b), hi(a) hi(b)): bf16 operands, fp32 products and
@@ -84,25 +85,36 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-// Warp-wide TMA load of one chunk: keys [y, y + 64) of kv-head z, K into
-// dst[0, 16K) and V into dst[16K, 32K), each as two 64-column 128B-swizzled
-// boxes.  Every lane calls it with the same operands; elect.sync picks the
-// lane that adds the 32 KB to `bar` and issues the four loads.
+// Warp-wide TMA load of one chunk: keys [y, y + 128) of kv-head z, K into
+// dst[0, 32K) and V into dst[32K, 64K).  Each of the two 64-column halves of K
+// (and of V) is 128 rows of 128 bytes, 128B-swizzled, loaded as two 64-row
+// boxes.  Every lane calls it with the same operands; elect.sync picks the lane
+// that adds the 64 KB to `bar` and issues the eight loads.
 __device__ __forceinline__ void tma_load_kv_chunk_warp(uint32_t dst, const void *tmap_k, const void *tmap_v,
                                                        uint32_t bar, int y, int z) {
     asm volatile(
-        "{\n\t.reg .pred e;\n\t"
+        "{\n\t.reg .pred e;\n\t.reg .b32 y1;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
-        "@e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%2], 32768;\n\t"
+        "add.s32 y1, %4, 64;\n\t"
+        "@e mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%2], 65536;\n\t"
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
         "[%0], [%1, {0, %4, %5}], [%2];\n\t"
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%6], [%1, {64, %4, %5}], [%2];\n\t"
+        "[%6], [%1, {0, y1, %5}], [%2];\n\t"
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%7], [%3, {0, %4, %5}], [%2];\n\t"
+        "[%7], [%1, {64, %4, %5}], [%2];\n\t"
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%8], [%3, {64, %4, %5}], [%2];\n\t}\n" ::"r"(dst),
-        "l"(tmap_k), "r"(bar), "l"(tmap_v), "r"(y), "r"(z), "r"(dst + 8192), "r"(dst + 16384), "r"(dst + 24576)
+        "[%8], [%1, {64, y1, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%9], [%3, {0, %4, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%10], [%3, {0, y1, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%11], [%3, {64, %4, %5}], [%2];\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%12], [%3, {64, y1, %5}], [%2];\n\t}\n" ::"r"(dst),
+        "l"(tmap_k), "r"(bar), "l"(tmap_v), "r"(y), "r"(z), "r"(dst + 8192), "r"(dst + 16384), "r"(dst + 24576),
+        "r"(dst + 32768), "r"(dst + 40960), "r"(dst + 49152), "r"(dst + 57344)
         : "memory");
 }
 
@@ -112,8 +124,8 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     const uint32_t ring = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kDiagStages * kChunkBytes);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kDiagStages);
-    // per stage: bit u set iff key (chunk start + u) is a vertical key (written by the
-    // producer before it arrives on the stage's full barrier)
+    // per stage: bit u of its two words set iff key (chunk start + u) is a vertical key
+    // (written by the producer before it arrives on the stage's full barrier)
     uint64_t *vmask = bars + 2 * kDiagStages + 1;
     auto full_bar = [&](int s) { return smem_u32(bars + s); };
     auto empty_bar = [&](int s) { return smem_u32(bars + kDiagStages + s); };
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                 const int gx = __shfl_sync(0xffffffffu, gwin.x, gi & 31), gy = __shfl_sync(0xffffffffu, gwin.y, gi & 31);
                 if (gx > rmax) break;  // groups ascend: no row of this tile reaches the rest
                 const int a = max(0, r0 - gy), b = rmax - gx;
-                const int nc = (b - a + kHalf) / kHalf;
+                const int nc = (b - a + kChunkKeys) / kChunkKeys;
                 for (int j = 0; j < nc; ++j, ++c) {
                     const int s = c % kDiagStages;
                     const bool got = wait_bounded_sleep(empty_bar(s), ((c / kDiagStages) & 1) ^ 1, wc, wait_site(8, s, c));
@@ -168,9 +180,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                         ok = false;
                         break;
                     }
-                    tma_load_kv_chunk_warp(ring + s * kChunkBytes, &P.tmap_k, &P.tmap_v, full_bar(s), a + j * kHalf,
-                                           g);
-                    if (lane == 0) vmask[s] = bits64_at(bv, P.n >> 5, a + j * kHalf);
+                    tma_load_kv_chunk_warp(ring + s * kChunkBytes, &P.tmap_k, &P.tmap_v, full_bar(s),
+                                           a + j * kChunkKeys, g);
+                    if (lane == 0) {
+                        vmask[2 * s] = bits64_at(bv, P.n >> 5, a + j * kChunkKeys);
+                        vmask[2 * s + 1] = bits64_at(bv, P.n >> 5, a + j * kChunkKeys + 64);
+                    }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full_bar(s));
                 }
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
     const int r = rw + (lane & 15);     // query row in the tile
     const int hf = lane >> 4;           // head-dimension half
     const float sl2 = P.scale_log2;
-    const uint32_t kbase = ring + hf * 8192;  // this thread's K box of a stage; its V box is 16 KB further
+    const uint32_t kbase = ring + hf * 16384;  // this thread's K half of a stage; its V half is 32 KB further
     const uint32_t *vmask32 = reinterpret_cast<const uint32_t *>(vmask);
     int win_lo = -1, st_lo = 0;  // first chunk of the current window and its stage
     int c_base = 0;  // sequence number of the current group's first chunk
@@ -267,7 +282,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
             G.w = __shfl_sync(0xffffffffu, gwin.w, gi & 31);
             if (G.x > rmax) break;
             const int a = max(0, r0 - G.y), b = rmax - G.x;
-            const int nc = (b - a + kHalf) / kHalf;
+            const int nc = (b - a + kChunkKeys) / kChunkKeys;
             // offsets of the group from the largest down (the key ranges move forward),
             // 32 at a time: lane l holds the l-th of the batch, broadcast by shuffle (a
             // lone offset is the descriptor's own first offset: nothing to load)
@@ -279,7 +294,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                     const int u0 = r0 - off - a;  // range position of row 0's key
                     const int ulo = max(0, u0 + rw), uhi = min(u0 + rw + 15, u0 + last_r);
                     if (ulo > uhi) continue;  // no valid row of this warp meets a key of this offset
-                    const int clo = c_base + (ulo >> 6), chi = c_base + (uhi >> 6);
+                    const int clo = c_base + (ulo >> 7), chi = c_base + (uhi >> 7);
                     if (clo != win_lo || chi >= got) {  // the window moved: release below it, see it full
                         if (!need(clo, chi)) {
                             ok = false;
@@ -292,11 +307,11 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                     const bool in = row_ok && u >= 0;
                     const int uc = max(u, 0);
                     // the row's chunk is the window's first or second (the 16 rows span at most two)
-                    int st = st_lo + ((uc >> 6) - (ulo >> 6));
+                    int st = st_lo + ((uc >> 7) - (ulo >> 7));
                     if (st >= kDiagStages) st -= kDiagStages;
-                    const int ur = uc & 63;
+                    const int ur = uc & 127;
                     // in the mask unless the key is a vertical (those are the tile kernel's)
-                    const bool use = in && !((vmask32[2 * st + (ur >> 5)] >> (ur & 31)) & 1u);
+                    const bool use = in && !((vmask32[4 * st + (ur >> 5)] >> (ur & 31)) & 1u);
                     // row ur of the stage; its 16-byte chunk i sits at chunk i ^ (ur & 7) (128B swizzle)
                     const uint32_t ka = kbase + (uint32_t)st * kChunkBytes + (uint32_t)ur * 128 + ((ur & 7) << 4);
                     float s = 0.f;
@@ -330,7 +345,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                         const uint16_t pb = bf16_bits(p);  // P enters P V in bf16, as on the tensor cores
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const uint4 vvi = lds128((ka + 16384) ^ (i << 4));
+                            const uint4 vvi = lds128((ka + 32768) ^ (i << 4));
                             axpy2_bf16(vvi.x, pb, o[8 * i], o[8 * i + 1]);
                             axpy2_bf16(vvi.y, pb, o[8 * i + 2], o[8 * i + 3]);
                             axpy2_bf16(vvi.z, pb, o[8 * i + 4], o[8 * i + 5]);
