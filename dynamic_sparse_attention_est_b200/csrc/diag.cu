@@ -314,8 +314,12 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                     const bool use = in && !((vmask32[4 * st + (ur >> 5)] >> (ur & 31)) & 1u);
                     // row ur of the stage; its 16-byte chunk i sits at chunk i ^ (ur & 7) (128B swizzle)
                     const uint32_t ka = kbase + (uint32_t)st * kChunkBytes + (uint32_t)ur * 128 + ((ur & 7) << 4);
-                    float s = 0.f;
-                    if (use) {
+                    float s;
+                    // no branch on `use`: every lane computes, and a lane outside the mask
+                    // adds P = 0.  Its address always lies in the ring: rows inside the tile read
+                    // a chunk of the window (real, finite K and V); rows past the tile's end may
+                    // read the stage after it, and their state is never stored.
+                    {
                         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight chains of 8
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -339,8 +343,8 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                         l *= alpha;
                         m = grow ? x : m;
                     }
-                    if (use) {
-                        const float p = ex2_approx(x - m);
+                    {
+                        const float p = use ? ex2_approx(x - m) : 0.f;
                         l += p;
                         const uint16_t pb = bf16_bits(p);  // P enters P V in bf16, as on the tensor cores
 #pragma unroll
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kDiagThreads, 1) vs_diag_kernel(const __grid_c
                             axpy2_bf16(vvi.z, pb, o[8 * i + 4], o[8 * i + 5]);
                             axpy2_bf16(vvi.w, pb, o[8 * i + 6], o[8 * i + 7]);
                         }
-                        ++pairs;  // counted by both threads of the row, halved at the end
+                        pairs += use ? 1u : 0u;  // counted by both threads of the row, halved at the end
                     }
                 }
             }
