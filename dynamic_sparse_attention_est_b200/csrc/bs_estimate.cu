@@ -13,8 +13,9 @@
 //           size (split-bf16 products in the manner of Henry, Tang and Heinecke,
 //           "Leveraging the bfloat16 artificial intelligence datatype for
 //           higher-precision computations", 2019), smallest first;
-//   top-k   diagonal block i always kept, the best topk-1 of j < i by radix
-//           select (ties to the lower j), ascending.
+//   top-k   diagonal block i always kept, the best topk-1 of j < i (ties to
+//           the lower j), ascending: a histogram of value bins finds the
+//           threshold bin, an exact selection settles it.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
