@@ -76,24 +76,28 @@ def parse():
     return a
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
-# launch, from the ncu capture summarised in profiles/, valid only for the
-# attention source it was taken on (sha1 of csrc/attention.cu).
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
+# kernel on a workload, from the ncu captures summarised in profiles/ (taken on
+# that workload's own bench command), valid only for the source it was taken
+# on (sha1 of the kernel's file).
 TRAFFIC = {
-    "vs-gqa-32k": ("3f22d096b5042b08e8f74f0b3b6f3dc29b4de356", 3.393959e9 + 0.241058e9),
+    ("attn_kernel<VS>", "vs-gqa-32k"): ("attention.cu", "3f22d096b5042b08e8f74f0b3b6f3dc29b4de356",
+                                        3.393959e9 + 0.241058e9),
+    ("vs_diag_kernel", "vs-1h-1m"): ("diag.cu", "1c46171e2aa10929f6a120b36237fe141ac0255b",
+                                     197.478696e9 + 0.548004e9),
 }
 
 
-def attention_traffic(workload: str):
+def kernel_traffic(kernel: str, workload: str):
     import hashlib
 
-    entry = TRAFFIC.get(workload) if workload else None
+    entry = TRAFFIC.get((kernel, workload)) if workload else None
     if entry is None:
         return None
-    src = os.path.join(ROOT, "dynamic_sparse_attention_est_b200", "csrc", "attention.cu")
+    src = os.path.join(ROOT, "dynamic_sparse_attention_est_b200", "csrc", entry[0])
     with open(src, "rb") as f:
         sha = hashlib.sha1(f.read()).hexdigest()
-    return entry[1] if sha == entry[0] else None
+    return entry[2] if sha == entry[1] else None
 
 
 def pick_bf16_peak(peaks, elapsed_ms, clk):
@@ -143,7 +147,7 @@ def kernel_rooflines(kernels, detail, peaks, src, peak, peak_key, elapsed, clk, 
             ach = flops / sec / 1e12
             return {"kernel": name, "bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
                     "frac": round(ach / peak, 4), "flops_per_launch": flops,
-                    "traffic": attention_traffic(traffic_key) if name == "attn_kernel<VS>" else None,
+                    "traffic": kernel_traffic(name, traffic_key),
                     "ms_per_launch": k["ms_per_launch"],
                     "peak_source": f"{src} {peak_key} (timed region {elapsed:.0f} ms, median SM clock "
                                    f"{clk.get('sm_mhz')} MHz)"}
@@ -152,7 +156,8 @@ def kernel_rooflines(kernels, detail, peaks, src, peak, peak_key, elapsed, clk, 
             ach = flops / sec / 1e12
             pk = alu_peak_tflops(peaks.get("sm_max_mhz") or 1965.0)
             return {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(pk, 1),
-                    "unit": "TFLOP/s", "frac": round(ach / pk, 4), "flops_per_launch": flops, "traffic": None,
+                    "unit": "TFLOP/s", "frac": round(ach / pk, 4), "flops_per_launch": flops,
+                    "traffic": kernel_traffic(name, traffic_key),
                     "ms_per_launch": k["ms_per_launch"],
                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x max SM clock"}
         return {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,

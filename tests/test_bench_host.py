@@ -35,10 +35,13 @@ def test_parse_defaults_and_options(monkeypatch):
 
 
 def test_traffic_only_for_the_captured_source():
-    assert bench.attention_traffic(None) is None
-    assert bench.attention_traffic("no-such-workload") is None
-    v = bench.attention_traffic("vs-gqa-32k")
-    assert v is None or v > 0
+    assert bench.kernel_traffic("attn_kernel<VS>", None) is None
+    assert bench.kernel_traffic("attn_kernel<VS>", "no-such-workload") is None
+    assert bench.kernel_traffic("vs_diag_kernel", "mixed-gqa-1m") is None  # not captured there
+    for kernel, workload in (("attn_kernel<VS>", "vs-gqa-32k"), ("vs_diag_kernel", "vs-1h-1m")):
+        v = bench.kernel_traffic(kernel, workload)
+        assert v is None or v > 0  # None once the kernel's source differs from the captured one
+
 
 
 def test_tile_flops():
